@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Decode benchmark: sparse-attention layer-steps/s at 32K context on B200.
+
+Workload: a Llama-3.1-8B-shaped attention layer (32 query / 8 KV heads,
+head_dim 128, batch 1, 32768-token paged bf16 cache, block sizes per KV head
+drawn from {16, 32, 64} with probabilities {0.25, 0.25, 0.5}, token budget
+2048, INT4 centroids).  One benchmark step decodes one token through
+`--layers` (default 64) such layers, each with its own cache, centroids and
+query, so the working set (8 GiB) is far larger than L2.  Each layer-step is
+one absp_decode_step launch; the layer-steps of a step are captured in a
+CUDA graph and every launch waits for the previous one to finish before it
+reads anything (programmatic dependent launch only overlaps the launch
+latency), as consecutive layers of a real decode would.
+
+value   = layer-steps/s over all ranks (weak scaling: every rank decodes its
+          own layer stack, no collective on the data path);
+e2e     = the same through absp_decode_step_host (query copied from pinned
+          host memory and output copied back inside every layer-step);
+roofline= algorithmic bytes of a layer-step (centroid codes + per-channel
+          parameters + valid selected K/V rows + q and out) / average launch
+          time, against the measured HBM copy bandwidth;
+rebuild = centroid build + INT4 quantisation of every layer (steps 1-2),
+          timed separately (it runs once per cache, not per token).
+
+`--impl reference` times the CPU oracle on the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn decode layer-steps/s at 32K ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "layer-steps/s"
+WORKLOAD = "llama31_8b_32k"
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "block_sparse_attention_kv_b200", "csrc", f)
+                  for f in ("decode.cu", "absp_internal.cuh")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="absp", choices=["absp", "reference"])
+    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------- helpers --
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, index: int, period: float = 0.005):
+        super().__init__(daemon=True)
+        self.index, self.period = index, period
+        self.sm, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def run(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.sm.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        self.join(timeout=2)
+        if not self.sm:
+            return None
+        return {"sm_mhz": float(statistics.median(self.sm)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.sm), "reasons": sorted(self.reasons)}
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """ncu DRAM bytes per launch, if recorded for the current kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        if rec.get("source_sha") == kernel_source_hash():
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def step_bytes(d, sel, cnt):
+    """Algorithmic bytes of one decode layer-step of layer data `d`."""
+    lens = d.seq_lens.cpu().numpy()
+    S, Hkv, Hq = d.num_seqs, d.num_kv_heads, d.num_q_heads
+    total = S * Hq * 128 * 2 * 2                       # q in + out
+    for s in range(S):
+        L = int(lens[s])
+        for h in range(Hkv):
+            bs = int(d.block_size[h])
+            n = (L + bs - 1) // bs
+            total += n * 64 + 128 * 8                  # codes + scale/zp
+            toks = 0
+            for b in sel[s, h, :cnt[s, h]]:
+                toks += min(bs, L - int(b) * bs)
+            total += toks * 2 * 128 * 2                # K and V rows
+    return total
+
+
+def rebuild_bytes(d):
+    lens = d.seq_lens.cpu().numpy()
+    tot = 0
+    for s in range(d.num_seqs):
+        L = int(lens[s])
+        for h in range(d.num_kv_heads):
+            bs = int(d.block_size[h])
+            tot += L * 256 + ((L + bs - 1) // bs) * 64 + 128 * 8
+    return tot
+
+
+# ------------------------------------------------------- CPU oracle leg --
+
+def oracle_layer_sample(layer_index: int = 0):
+    """Host copy of one layer plus the oracle's prebuilt centroids."""
+    from block_sparse_attention_kv_b200 import synth
+    from oracle import absp_oracle as O
+    w = synth.WORKLOADS[WORKLOAD]
+    d = synth.make_layer(w, layer_index, "cpu")
+    hl = synth.host_layer(d)
+    prep = []
+    for s in range(hl.q_bits.shape[0]):
+        qf = O.decode_bf16(hl.q_bits[s])
+        for h in range(len(hl.block_size)):
+            keys, vals = O.head_keys_values(hl, s, h)
+            bs = int(hl.block_size[h])
+            chat = O.dequantize(O.quantize_centroids(O.build_centroids(keys, bs)))
+            prep.append((qf, h, chat, keys, vals, bs, int(hl.seq_lens[s])))
+    G = hl.q_bits.shape[1] // len(hl.block_size)
+    return prep, G, int(hl.budget)
+
+
+def time_oracle(prep, G, budget, steps: int = None, seconds: float = None):
+    """Runs oracle decode (steps 3-5) over (seq, head) units; returns
+    (units done, elapsed s)."""
+    from oracle import absp_oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except Exception:
+        lim = None
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        if steps is not None and done >= steps:
+            break
+        if seconds is not None and time.perf_counter() - t0 >= seconds:
+            break
+        qf, h, chat, keys, vals, bs, L = prep[done % len(prep)]
+        O.decode_head(qf, h, G, chat, keys, vals, bs, L, budget)
+        done += 1
+    el = time.perf_counter() - t0
+    if lim is not None:
+        lim.unregister() if hasattr(lim, "unregister") else None
+    return done, el
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    prep, G, budget = oracle_layer_sample(0)
+    units_per_layer_step = len(prep)
+    time_oracle(prep, G, budget, steps=args.warmup)
+    done, el = time_oracle(prep, G, budget, steps=args.steps)
+    layer_steps = done / units_per_layer_step
+    value = layer_steps / el
+    sample = (f"{args.steps} steps, each the oracle's steps 3-5 (score, top-K, "
+              f"attention) for one (sequence, KV head) of a {WORKLOAD} layer "
+              f"(1/{units_per_layer_step} layer-step), numpy fp64, 1 thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / max(done, 1) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "step": "one (sequence, KV head) decode unit"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------- GPU arm --
+
+def gpu_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from block_sparse_attention_kv_b200 import build as absp_build
+    if rank == 0 or world == 1:
+        absp_build.build()
+    if dist is not None:
+        dist.barrier()
+    from block_sparse_attention_kv_b200 import abi, pipeline, synth
+
+    w = synth.WORKLOADS[WORKLOAD]
+    L = args.layers
+    stream = torch.cuda.Stream(device=dev)
+    layers = []
+    with torch.cuda.stream(stream):
+        for i in range(L):
+            d = synth.make_layer(w, rank * L + i, dev)
+            layers.append(pipeline.DeviceLayer(d, stream=stream.cuda_stream))
+    stream.synchronize()
+
+    # steps 1-2 for every layer, timed (once per cache)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ws_n = max(abi.absp_build_workspace_size(x.kv) for x in layers)
+    bws = abi.alloc_workspace(ws_n, dev)
+    sc = stream.cuda_stream
+    for x in layers[:2]:                               # warm-up
+        abi.absp_build_centroids(x.kv, bws, sc)
+        abi.absp_quantize_centroids(x.kv, bws, x.cent, sc)
+    stream.synchronize()
+    ev0.record(stream)
+    for x in layers:
+        abi.absp_build_centroids(x.kv, bws, sc)
+        abi.absp_quantize_centroids(x.kv, bws, x.cent, sc)
+    ev1.record(stream)
+    stream.synchronize()
+    rebuild_ms = ev0.elapsed_time(ev1) / L
+    st, _ = abi.absp_check_device_error(bws, sc)
+    assert st == abi.ABSP_OK, "device fault while building centroids"
+    rb_bytes = sum(rebuild_bytes(x.data) for x in layers) / L
+    del bws
+
+    # algorithmic bytes from each layer's own selection
+    nbytes = []
+    for x in layers:
+        x.score_select()
+        stream.synchronize()
+        nbytes.append(step_bytes(x.data, x.sel.cpu().numpy(), x.sel_count.cpu().numpy()))
+        x.decode_step()                                # warm: attributes, occupancy
+    stream.synchronize()
+    for x in layers:
+        x.check()
+    bytes_per_launch = float(np.mean(nbytes))
+
+    # CUDA graph of one step = L layer-steps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for x in layers:
+            abi.absp_decode_step(x.kv, x.cent, x.data.q, x.budget, x.out, x.ws, sc)
+    stream.synchronize()
+
+    def timed(graph, steps, warm):
+        for _ in range(warm):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    with torch.cuda.stream(stream):
+        sampler = ClockSampler(local)
+        sampler.start()
+        ms = timed(g, args.steps, args.warmup)
+        clocks = sampler.stop()
+    for x in layers:
+        x.check()
+
+    e2e = None
+    if not args.no_e2e:
+        q_host = [x.data.q.cpu().pin_memory() for x in layers]
+        o_host = [torch.empty_like(q).pin_memory() for q in q_host]
+        g2 = torch.cuda.CUDAGraph()
+        for x, qh, oh in zip(layers, q_host, o_host):   # warm outside capture
+            abi.absp_decode_step_host(x.kv, x.cent, qh, x.budget, oh, x.ws, sc)
+        stream.synchronize()
+        with torch.cuda.graph(g2, stream=stream):
+            for x, qh, oh in zip(layers, q_host, o_host):
+                abi.absp_decode_step_host(x.kv, x.cent, qh, x.budget, oh, x.ws, sc)
+        with torch.cuda.stream(stream):
+            ms_e2e = timed(g2, args.steps, args.warmup)
+        for x, oh in zip(layers, o_host):
+            assert torch.equal(oh.view(torch.int16), x.out.cpu().view(torch.int16))
+        qb = sum(q.numel() * 2 for q in q_host)
+        e2e = {"value": world * L * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": qb, "d2h_bytes_per_step": qb,
+               "ms_per_step": ms_e2e / args.steps}
+        del g2
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        prep, G, budget = oracle_layer_sample(0)
+        done, el = time_oracle(prep, G, budget, seconds=args.cpu_seconds)
+        cpu = {"value": (done / len(prep)) / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{done} (sequence, KV head) decode units of one {WORKLOAD} layer "
+                         f"({done / len(prep):.2f} layer-steps, steps 3-5 from prebuilt "
+                         f"centroids), numpy fp64, 1 thread, {el:.1f} s"}
+
+    peak, peak_kind = hbm_peak()
+    launch_ms = ms / (args.steps * L)
+    achieved = bytes_per_launch / (launch_ms * 1e-3) / 1e9
+    traffic = recorded_traffic()
+    line = {
+        "metric": METRIC,
+        "value": world * L * args.steps / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": (f"{WORKLOAD}: Llama-3.1-8B-shaped attention layer decode, 32 q / 8 kv "
+                         f"heads, head_dim 128, batch 1, ctx 32768, budget 2048 tokens, "
+                         f"block sizes per kv head from {{16,32,64}}, INT4 centroids"),
+            "layers_per_step": L,
+            "step": f"one decode token through {L} layers with distinct caches",
+            "l2": f"inputs larger than L2: {L} distinct layer caches (~{L * 128 // 1024} GiB)",
+            "launch": "CUDA graph of fused score/select/attend launches, PDL",
+            "parallelism": f"dp{world} (independent layer stacks per GPU)",
+        },
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} HBM copy bandwidth",
+                     "kernel": "decode_kernel<full>",
+                     "bytes_per_launch": bytes_per_launch, "launch_us": launch_ms * 1e3},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": L * args.steps,
+        "clocks": clocks,
+        "rebuild": {"ms_per_layer": rebuild_ms, "bytes_per_layer": rb_bytes,
+                    "achieved_gbs": rb_bytes / (rebuild_ms * 1e-3) / 1e9,
+                    "frac": rb_bytes / (rebuild_ms * 1e-3) / 1e9 / peak},
+    }
+    del g
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+/*
+ * absp.h -- C ABI of the adaptive-block sparse decode attention library
+ * (libabsp.so, CUDA, sm_100a).
+ *
+ * The method is AB-Sparse: Sparse Attention with Adaptive Block Size
+ * (arXiv 2605.12110).  Its decode path, as its review page describes it:
+ *   - Fig. 1: keys are grouped into blocks; each block is represented by a
+ *     centroid; a query-centroid dot product scores each block; the top-K
+ *     blocks are selected; attention runs over their keys only.
+ *   - Fig. 3 / Fig. 5: each KV head has its own block size in {16, 32, 64},
+ *     fixed offline, so centroids are built once over all keys.
+ *   - Fig. 8 / abstract: centroids are kept as INT4 codes, asymmetric,
+ *     with per-channel parameters.
+ *   - Fig. 9: logical blocks are runs of consecutive 16-token physical
+ *     pages (block size / 16 pages per block); every head reads the same
+ *     number of pages, i.e. the budget is in tokens.
+ *
+ * Conventions shared by every call:
+ *   - All buffers are owned by the caller.  Pointers marked "device" must
+ *     be device memory of the current CUDA device; "host" means host memory.
+ *     The library never allocates device memory.
+ *   - Every call that launches work is asynchronous on `stream` (a
+ *     cudaStream_t passed as void*; NULL is the legacy default stream).
+ *   - Host-side argument checks return an error status before anything is
+ *     launched.  Faults detected on the device (a page id or block index
+ *     out of range, a length beyond the page table, a wait that timed out)
+ *     are recorded in the first bytes of the workspace and reported by
+ *     absp_check_device_error(); kernels never trap.
+ *   - head_dim must be 128 and page_size 16 (ABSP_ERR_UNSUPPORTED otherwise).
+ *   - No call throws; every call returns an absp_status.
+ */
+#ifndef ABSP_H_
+#define ABSP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ABSP_API __attribute__((visibility("default")))
+#else
+#define ABSP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t absp_status;
+#define ABSP_OK 0
+#define ABSP_ERR_INVALID_ARG 1   /* null pointer, bad size, misalignment   */
+#define ABSP_ERR_UNSUPPORTED 2   /* head_dim != 128, page_size != 16, ... */
+#define ABSP_ERR_CUDA 3          /* a CUDA runtime call failed            */
+#define ABSP_ERR_DEVICE_FAULT 4  /* a device-side bounds check fired      */
+#define ABSP_ERR_TIMEOUT 5       /* a device-side bounded wait gave up    */
+
+#define ABSP_HEAD_DIM 128
+#define ABSP_PAGE_SIZE 16
+#define ABSP_CODE_ROW_BYTES 64           /* 128 INT4 codes per centroid    */
+#define ABSP_MAX_KV_HEADS 64
+#define ABSP_MAX_GROUP 16                /* query heads per KV head        */
+#define ABSP_MAX_BLOCKS_PER_HEAD 16384   /* centroid rows per (seq, head)  */
+#define ABSP_MAX_BUDGET 65536            /* token budget per KV head       */
+
+/* One attention layer's paged KV cache (Fig. 9: physical pages, logical
+ * blocks).  Token t of sequence s lives in physical page
+ * page_table[s * max_pages_per_seq + t / 16], slot t % 16.  A page holds all
+ * KV heads: k_pages[page][kv_head][slot][channel], bf16, so one
+ * (page, head) slice is 4 KiB contiguous.  Query head j belongs to KV head
+ * j / (num_q_heads / num_kv_heads) (contiguous GQA grouping). */
+typedef struct absp_layer_kv {
+    int32_t num_seqs;            /* S >= 1                                  */
+    int32_t num_q_heads;         /* Hq, a multiple of Hkv, Hq/Hkv <= 16     */
+    int32_t num_kv_heads;        /* Hkv, 1..64                              */
+    int32_t head_dim;            /* must be 128                             */
+    int32_t page_size;           /* must be 16                              */
+    int32_t max_pages_per_seq;   /* page-table row stride (>= 1)            */
+    int64_t num_phys_pages;      /* pages in k_pages / v_pages (>= 1)       */
+    const int32_t* seq_lens;     /* device [S]; 0 <= len <= 16*max_pages    */
+    const int32_t* page_table;   /* device [S][max_pages_per_seq]           */
+    const void* k_pages;         /* device bf16, 256-byte aligned           */
+    const void* v_pages;         /* device bf16, 256-byte aligned           */
+    const int32_t* block_size;   /* HOST [Hkv], each 16, 32 or 64           */
+} absp_layer_kv;
+
+/* INT4 centroid store of one layer (Fig. 8: asymmetric, per channel).
+ * Head h of sequence s has capacity cap_h = ceil(16*max_pages_per_seq/bs_h)
+ * rows; its rows start at row  s * rows_per_seq + base_h  where
+ * base_h = sum_{h' < h} cap_h' and rows_per_seq = sum_h cap_h (see
+ * absp_centroid_row_offset).  Row b (block b of the head) holds 64 bytes:
+ * channel 2i in the low nibble of byte i, channel 2i+1 in the high nibble.
+ * Dequantised centroid = (code - zp[s][h][c]) * scale[s][h][c]. */
+typedef struct absp_centroids {
+    uint8_t* codes;              /* device, 256-byte aligned               */
+    float* scale;                /* device [S][Hkv][128]                   */
+    int32_t* zp;                 /* device [S][Hkv][128]                   */
+} absp_centroids;
+
+/* Human-readable name of a status code (static string, never NULL). */
+ABSP_API const char* absp_status_string(absp_status status);
+
+/* Bytes of the three centroid buffers for `kv` (host only, no launch). */
+ABSP_API absp_status absp_centroid_sizes(const absp_layer_kv* kv, size_t* codes_bytes,
+                                size_t* scale_bytes, size_t* zp_bytes);
+
+/* First code row of (seq, kv_head) in absp_centroids.codes (host only). */
+ABSP_API absp_status absp_centroid_row_offset(const absp_layer_kv* kv, int32_t seq,
+                                     int32_t kv_head, int64_t* row);
+
+/* Workspace bytes for absp_build_centroids + absp_quantize_centroids:
+ * 256 B header + per-channel min/max + fp64 centroids (1 KiB per row). */
+ABSP_API absp_status absp_build_workspace_size(const absp_layer_kv* kv, size_t* bytes);
+
+/* Workspace bytes for the decode calls (score/select, sparse decode,
+ * decode step, and the host-buffer decode step). */
+ABSP_API absp_status absp_decode_workspace_size(const absp_layer_kv* kv,
+                                       int32_t budget_tokens, size_t* bytes);
+
+/* Row stride of the block-index list `sel`: max over heads of
+ * K_h = max(1, budget / bs_h) (Fig. 9 equal token budget). */
+ABSP_API absp_status absp_select_capacity(const absp_layer_kv* kv, int32_t budget_tokens,
+                                 int32_t* kmax);
+
+/* Zero-fill a workspace (its error word must start at 0).  Call once per
+ * workspace before its first use. */
+ABSP_API absp_status absp_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Step 1 (Fig. 1 "block representation", Fig. 5 "centroids over all key
+ * vectors"): for every (seq, kv_head, block b) the mean of the block's
+ * valid keys, c[b][ch] = (sum_t K[t][ch]) / cnt_b, summed in token order in
+ * fp64 (a ragged last block averages its valid tokens only).  Writes the
+ * fp64 centroids and the per-channel min/max into `ws` (size from
+ * absp_build_workspace_size).  Reads every key of the layer once. */
+ABSP_API absp_status absp_build_centroids(const absp_layer_kv* kv, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* Step 2 (Fig. 8: INT4 asymmetric per-channel): from the workspace filled by
+ * absp_build_centroids, per (seq, kv_head, channel):
+ *   scale = fp32((max - min) / 15), zp = rint(-min / scale) (int32, not
+ *   clamped to 4 bits), code = clamp(rint(c / scale) + zp, 0, 15),
+ * rint = round half to even, all in fp64 except the stored scale; a channel
+ * with max == min gets scale 0, zp 0, codes 0.  Writes `out`. */
+ABSP_API absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws,
+                                    size_t ws_bytes, const absp_centroids* out,
+                                    void* stream);
+
+/* Steps 3-4 (Fig. 1 "dot product estimation", "importance score",
+ * "top-K selection"): for every (seq, kv_head), qbar = sum of the GQA
+ * group's queries (q: device bf16 [S][Hq][128]), score[b] =
+ * sum_ch qbar[ch] * (code[b][ch] - zp[ch]) * scale[ch] (fp32), then the
+ * K_h = min(n_h, max(1, budget / bs_h)) highest scores, ties to the lower
+ * block index.  Writes sel[(s*Hkv + h) * kmax + i], i < K_h, ascending
+ * block indices (kmax from absp_select_capacity), and sel_count[s*Hkv + h]
+ * = K_h.  sel: device int32 [S][Hkv][kmax]; sel_count: device int32
+ * [S][Hkv]. */
+ABSP_API absp_status absp_score_select(const absp_layer_kv* kv, const absp_centroids* cent,
+                              const void* q, int32_t budget_tokens, int32_t* sel,
+                              int32_t* sel_count, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Step 5 (Fig. 1 "sparse attention"): for every query head j of KV head h,
+ * out[s][j] = softmax_t(q_j . K_t / sqrt(128)) V over the valid tokens of
+ * the blocks listed in sel / sel_count (layout as written by
+ * absp_score_select for the same budget_tokens), gathered through the page
+ * table.  bf16 in, fp32 accumulation, bf16 out (device [S][Hq][128]).  A
+ * head with no valid token gets a zero output.  Block indices out of range
+ * are skipped and reported as ABSP_ERR_DEVICE_FAULT. */
+ABSP_API absp_status absp_sparse_decode(const absp_layer_kv* kv, const void* q,
+                               const int32_t* sel, const int32_t* sel_count,
+                               int32_t budget_tokens, void* out, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Steps 3-5 in one launch: score, select and attend, with the selection
+ * kept on chip.  Same results as absp_score_select followed by
+ * absp_sparse_decode. */
+ABSP_API absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centroids* cent,
+                             const void* q, int32_t budget_tokens, void* out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* absp_decode_step with HOST query and output buffers: copies q_host
+ * (bf16 [S][Hq][128], pinned for true asynchrony) into the workspace, runs
+ * the step and copies the result back to out_host, all on `stream`.  The
+ * caller synchronises `stream` before reading out_host. */
+ABSP_API absp_status absp_decode_step_host(const absp_layer_kv* kv,
+                                  const absp_centroids* cent, const void* q_host,
+                                  int32_t budget_tokens, void* out_host, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads the workspace's error word and clears it.
+ * Returns ABSP_OK, ABSP_ERR_DEVICE_FAULT or ABSP_ERR_TIMEOUT; *detail (if
+ * not NULL) receives the first faulting sequence/unit index. */
+ABSP_API absp_status absp_check_device_error(void* ws, size_t ws_bytes, void* stream,
+                                    int32_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ABSP_H_ */

@@ -252,6 +252,25 @@ def head_keys_values(layer, s, h):
     return keys, vals
 
 
+def decode_head(q_heads: np.ndarray, kv_head: int, group: int, chat: np.ndarray,
+                keys: np.ndarray, values: np.ndarray, bs: int, seq_len: int,
+                budget: int, sel_override=None):
+    """Steps 3-5 for one (sequence, KV head) from its (dequantised) centroids.
+
+    Returns (scores, k, sel, outputs [group][128]).
+    """
+    qbar = group_query(q_heads, kv_head, group)
+    sc = block_scores(chat, qbar)
+    k = min(blocks_per_head(budget, bs), chat.shape[0])
+    sel = select_blocks(sc, k)
+    use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)
+    toks = selected_tokens(use, bs, seq_len)
+    outs = np.zeros((group, HEAD_DIM), dtype=np.float64)
+    for i, j in enumerate(range(kv_head * group, (kv_head + 1) * group)):
+        outs[i] = attend(q_heads[j], keys, values, toks)
+    return sc, k, sel, outs
+
+
 def run_layer(layer, quantize: bool = True, sel_override=None,
               heads=None, with_attention: bool = True) -> LayerResult:
     """All five steps for every (sequence, KV head) of a host layer.
@@ -278,16 +297,10 @@ def run_layer(layer, quantize: bool = True, sel_override=None,
             cent = build_centroids(keys, bs)
             qc = quantize_centroids(cent)
             chat = dequantize(qc) if quantize else cent
-            qbar = group_query(qf, h, G)
-            sc = block_scores(chat, qbar)
-            k = min(blocks_per_head(layer.budget, bs), cent.shape[0])
-            sel = select_blocks(sc, k)
+            ov = None if sel_override is None else sel_override[(s, h)]
+            sc, k, sel, outs = decode_head(qf, h, G, chat, keys, vals, bs, L,
+                                           layer.budget, sel_override=ov)
             res.heads[(s, h)] = HeadResult(L, bs, cent, qc, sc, k, sel)
-            if not with_attention:
-                continue
-            use = sel if sel_override is None else \
-                np.asarray(sel_override[(s, h)], dtype=np.int64)
-            toks = selected_tokens(use, bs, L)
-            for j in range(h * G, (h + 1) * G):
-                res.out[s, j] = attend(qf[j], keys, vals, toks)
+            if with_attention:
+                res.out[s, h * G:(h + 1) * G] = outs
     return res

@@ -1,0 +1,125 @@
+"""C-ABI library: loads, exports every declared symbol, validates on the host.
+
+No test here launches device work: each call either is pure host logic or
+returns an argument error before any CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_kv_b200 import build as absp_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def abi():
+    absp_build.build()
+    from block_sparse_attention_kv_b200 import abi as m
+    return m
+
+
+def _declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "absp.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:ABSP_API\s+)?(?:absp_status|const char\*)\s+(absp_\w+)\(",
+                                 txt, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for want in ("absp_build_centroids", "absp_quantize_centroids", "absp_score_select",
+                 "absp_sparse_decode", "absp_decode_step"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(abi):
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(_declared_symbols()) == set(abi.EXPORTED)
+
+
+def _kv(abi, **over):
+    # fake (never dereferenced) device addresses, 256-byte aligned
+    args = dict(seq_lens=0x10000, page_table=0x20000, k_pages=0x100000,
+                v_pages=0x200000, block_size=[16, 64], num_q_heads=8,
+                num_phys_pages=512)
+    args.update(over)
+    kv = abi.LayerKV(None, None, None, None, args["block_size"], args["num_q_heads"],
+                     num_phys_pages=args["num_phys_pages"])
+    kv.c.num_seqs = over.get("num_seqs", 1)
+    kv.c.max_pages_per_seq = over.get("max_pages", 512)
+    kv.c.seq_lens = args["seq_lens"]
+    kv.c.page_table = args["page_table"]
+    kv.c.k_pages = args["k_pages"]
+    kv.c.v_pages = args["v_pages"]
+    kv.c.head_dim = over.get("head_dim", 128)
+    kv.c.page_size = over.get("page_size", 16)
+    return kv
+
+
+def test_sizes_follow_the_layout(abi):
+    kv = _kv(abi)
+    codes, scale, zp = abi.absp_centroid_sizes(kv)
+    # 8192 tokens: 512 rows at bs 16 + 128 rows at bs 64, 64 B each
+    assert codes == (512 + 128) * 64
+    assert scale == zp == 2 * 128 * 4
+    assert abi.absp_centroid_row_offset(kv, 0, 1) == 512
+    kv3 = _kv(abi, num_seqs=3)
+    assert abi.absp_centroid_row_offset(kv3, 2, 1) == 2 * 640 + 512
+    assert abi.absp_select_capacity(kv, 1024) == 64
+    assert abi.absp_select_capacity(kv, 40) == 2          # max(1, 40/16)
+    ws = abi.absp_build_workspace_size(kv)
+    assert ws == 256 + 2 * 2 * 128 * 8 + 640 * 128 * 8
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(head_dim=64), 2),
+    (dict(page_size=32), 2),
+    (dict(block_size=[16, 48]), 1),
+    (dict(num_q_heads=7), 1),
+    (dict(num_q_heads=2 * 17), 2),          # group of 17 > 16
+    (dict(k_pages=0x100010), 1),            # not 256-byte aligned
+    (dict(seq_lens=0), 1),
+])
+def test_invalid_layers_are_rejected(abi, over, status):
+    kv = _kv(abi, **over)
+    with pytest.raises(abi.AbspError) as e:
+        abi.absp_centroid_sizes(kv)
+    assert e.value.status == status
+
+
+def test_misaligned_pages_rejected_by_decode_calls(abi):
+    kv = _kv(abi, k_pages=0x100010)
+    with pytest.raises(abi.AbspError) as e:
+        abi.absp_build_centroids(kv, torch.zeros(1 << 20, dtype=torch.uint8))
+    assert e.value.status == abi.ABSP_ERR_INVALID_ARG
+
+
+def test_budget_limits(abi):
+    kv = _kv(abi)
+    for b in (0, 8, 15, 70000):
+        with pytest.raises(abi.AbspError) as e:
+            abi.absp_select_capacity(kv, b)
+        assert e.value.status == abi.ABSP_ERR_INVALID_ARG
+
+
+def test_small_workspace_rejected_before_launch(abi):
+    kv = _kv(abi)
+    tiny = torch.zeros(64, dtype=torch.uint8)
+    with pytest.raises(abi.AbspError) as e:
+        abi.absp_build_centroids(kv, tiny)
+    assert e.value.status == abi.ABSP_ERR_INVALID_ARG
+
+
+def test_null_layer_and_status_strings(abi):
+    lib = abi.lib()
+    assert lib.absp_centroid_sizes(None, None, None, None) == abi.ABSP_ERR_INVALID_ARG
+    assert abi.absp_status_string(0) == "ok"
+    assert "bounds" in abi.absp_status_string(abi.ABSP_ERR_DEVICE_FAULT)
+    assert abi.absp_status_string(99) == "unknown status"
