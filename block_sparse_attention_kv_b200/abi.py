@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 from ctypes import (POINTER, Structure, c_char_p, c_int32, c_int64, c_size_t,
-                    c_uint8, c_void_p)
+                    c_uint8, c_uint32, c_void_p)
 
 import numpy as np
 import torch
@@ -25,6 +25,8 @@ ABSP_ERR_UNSUPPORTED = 2
 ABSP_ERR_CUDA = 3
 ABSP_ERR_DEVICE_FAULT = 4
 ABSP_ERR_TIMEOUT = 5
+
+ABSP_STEP_EARLY_PREFETCH = 1
 
 HEAD_DIM = 128
 PAGE_SIZE = 16
@@ -87,6 +89,8 @@ def _load() -> ctypes.CDLL:
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
         "absp_decode_step": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
                                   c_void_p, c_void_p, c_size_t, c_void_p]),
+        "absp_decode_step_ex": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
+                                     c_void_p, c_void_p, c_size_t, c_uint32, c_void_p]),
         "absp_decode_step_host": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
         "absp_check_device_error": (st, [c_void_p, c_size_t, c_void_p, P(c_int32)]),
@@ -103,7 +107,8 @@ EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_row_offs
             "absp_build_workspace_size", "absp_decode_workspace_size",
             "absp_select_capacity", "absp_workspace_init", "absp_build_centroids",
             "absp_quantize_centroids", "absp_score_select", "absp_sparse_decode",
-            "absp_decode_step", "absp_decode_step_host", "absp_check_device_error")
+            "absp_decode_step", "absp_decode_step_ex", "absp_decode_step_host",
+            "absp_check_device_error")
 
 
 def lib() -> ctypes.CDLL:
@@ -272,6 +277,13 @@ def absp_decode_step(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
                      out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
     _check(_lib.absp_decode_step(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(out), _ptr(ws),
                                  ws.numel(), _stream(stream)), "absp_decode_step")
+
+
+def absp_decode_step_ex(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
+                        out: torch.Tensor, ws: torch.Tensor, flags: int, stream=None) -> None:
+    _check(_lib.absp_decode_step_ex(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(out), _ptr(ws),
+                                    ws.numel(), int(flags), _stream(stream)),
+           "absp_decode_step_ex")
 
 
 def absp_decode_step_host(kv: LayerKV, cent: Centroids, q_host: torch.Tensor, budget: int,

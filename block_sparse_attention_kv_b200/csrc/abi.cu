@@ -144,7 +144,7 @@ absp_status check_cent(const absp_centroids* c) {
 
 absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* cent,
                        const void* q, int32_t budget, int32_t* sel, int32_t* sel_count,
-                       void* out, void* ws, size_t ws_bytes, void* stream) {
+                       void* out, void* ws, size_t ws_bytes, void* stream, uint32_t flags = 0) {
     KvDesc d;
     absp_status st = make_desc(kv, &d, (mode & kModeAttend) != 0);
     if (st != ABSP_OK) return st;
@@ -180,7 +180,8 @@ absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* 
     a.budget = budget;
     a.err = static_cast<int32_t*>(ws);
     a.nmax = nmax;
-    return from_cuda(launch_decode(mode, a, &tmk, &tmv, use_pdl(),
+    const bool early = (flags & ABSP_STEP_EARLY_PREFETCH) != 0;
+    return from_cuda(launch_decode(mode, a, &tmk, &tmv, use_pdl(), early,
                                    static_cast<cudaStream_t>(stream)));
 }
 
@@ -295,6 +296,14 @@ absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centroids* cent
                              void* stream) {
     return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
                       stream);
+}
+
+absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
+                                const void* q, int32_t budget_tokens, void* out, void* ws,
+                                size_t ws_bytes, uint32_t flags, void* stream) {
+    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH)) != 0) return ABSP_ERR_INVALID_ARG;
+    return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
+                      stream, flags);
 }
 
 absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids* cent,

@@ -85,15 +85,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same wait with cluster-scope acquire: orders the distributed-shared-memory
+// writes of the CTAs that arrived remotely before reads that follow.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Arrive (release, cluster scope) on an mbarrier of another CTA of the
+// cluster; `remote` is a shared::cluster address from dsmem_addr().
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote)
+                 : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Wait for phase `parity` of an mbarrier, giving up after ~1 s.  On timeout
 // the error word records ABSP_ERR_TIMEOUT and the caller carries on (so that
 // every later cluster barrier is still reached); results are then garbage
 // and the host sees the error.
+template <bool CLUSTER_ACQUIRE = false>
 __device__ __forceinline__ void mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   int32_t* err, int where) {
-    if (mbar_try_wait(bar, parity)) return;
+    auto poll = [&] {
+        return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    };
+    if (poll()) return;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!poll()) {
         if (globaltimer_ns() - t0 > 1000000000ull) {
             set_error(err, ABSP_ERR_TIMEOUT, where);
             return;
@@ -156,6 +185,28 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
     return r;
 }
 
+// Asynchronous 16-byte store into a CTA of the cluster that completes 16
+// bytes of transaction count on that CTA's mbarrier `remote_bar` (both
+// shared::cluster addresses of the same destination CTA).
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float b, float c,
+                                            float d, uint32_t remote_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+        "[%5];" ::"r"(remote_addr),
+        "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+        : "memory");
+}
+
+// 8-byte variant of st_async_v4.
+__device__ __forceinline__ void st_async_v2(uint32_t remote_addr, float a, float b,
+                                            uint32_t remote_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+            remote_addr),
+        "f"(a), "f"(b), "r"(remote_bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
@@ -197,18 +248,20 @@ __device__ __forceinline__ void mma_bf16(float& d0, float& d1, float& d2, float&
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+#pragma nv_diag_suppress 550  // the discarded rows 8..15 below
 // Same tile op when rows 8..15 of A are zero (a GQA group of <= 8 heads):
 // only the accumulators of rows 0..7 are carried; rows 8..15 are written to
 // discarded temporaries and read as zero.
 __device__ __forceinline__ void mma_bf16_top(float& d0, float& d1, uint32_t a0, uint32_t a2,
                                              uint32_t b0, uint32_t b1) {
-    float x2, x3;
+    float x2, x3;  // rows 8..15: discarded
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %12};"
         : "=f"(d0), "=f"(d1), "=f"(x2), "=f"(x3)
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0), "f"(d1), "f"(0.0f));
 }
+#pragma nv_diag_default 550
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -249,7 +302,9 @@ struct DecodeArgs {
     int32_t* err;
     int32_t nmax;                 // bound on blocks per head for this layer
 };
+// early_prefetch: codes, parameters, lengths and page table are read before
+// the programmatic-dependency wait (only the query after it).
 cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
-                          const CUtensorMap* tmv, bool pdl, cudaStream_t st);
+                          const CUtensorMap* tmv, bool pdl, bool early_prefetch, cudaStream_t st);
 
 }  // namespace absp

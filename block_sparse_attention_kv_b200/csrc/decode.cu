@@ -8,23 +8,29 @@
 //   A  score:   CTA r streams its contiguous 1/C share of the head's code
 //               rows into shared memory with 1-D bulk copies, scores every
 //               row (8 lanes per 64-byte row, 16 codes per lane, fp32) and
-//               broadcasts each score into the score array of every CTA of
-//               the cluster through distributed shared memory.
-//   B  cluster barrier: every CTA now holds all n_h scores.
-//   C  select:  every CTA runs the same deterministic radix select (four
-//               8-bit digit passes over order-preserving uint32 keys, ties to
-//               the lower block index) and an ordered compaction, so all
-//               CTAs hold the same ascending block list without another
+//               sends each group of 4 scores to every CTA of the cluster
+//               with asynchronous 16-byte distributed-shared-memory stores
+//               that count down the receiver's mbarrier.  Meanwhile the
+//               sequence's page-table row is prefetched into L2.
+//   B  each CTA waits on its own mbarrier until all n_h scores arrived.
+//   C  select:  every CTA runs the same deterministic top-K (largest scores,
+//               ties to the lower block index): a 1024-bin histogram over the
+//               score range finds the bin holding the K-th score, the few
+//               scores in that bin are ranked exactly, and an ordered
+//               compaction writes the ascending block list.  A 4 x 8-bit
+//               radix select over order-preserving keys covers degenerate
+//               ranges.  All CTAs hold the same list without another
 //               exchange.
-//   D  attend:  the selected blocks expand to bs/16 pages each; CTA r takes
-//               a contiguous 1/C share of those pages and loads each
-//               (page, head) K and V slice with 2-D tensor copies (128-byte
-//               swizzle, no multicast).  Each warp owns one page per round:
-//               S^T = Q K^T and O += P V on mma.sync bf16 tiles with the GQA
-//               group as the 16-row M dimension, online softmax in fp32.
-//   E  merge:   warps merge in shared memory; CTAs merge their (m, l, O)
-//               partials into CTA 0 through distributed shared memory; CTA 0
-//               writes the bf16 output.
+//   D  attend:  the selected blocks expand to bs/16 pages each; CTA r takes a
+//               contiguous 1/C share of those pages.  Each warp owns every
+//               8th page: it loads the (page, head) K and V slices with 2-D
+//               tensor copies (128-byte swizzle, no multicast) on its own
+//               mbarrier, then computes S^T = Q K^T and O += P V on mma.sync
+//               bf16 tiles with the GQA group as the 16-row M dimension and an
+//               online softmax in fp32.
+//   E  merge:   warps merge in shared memory; CTAs write their (m, l, O)
+//               partials into CTA 0 through distributed shared memory and
+//               arrive on CTA 0's mbarrier; CTA 0 merges and writes bf16.
 // Modes: select only (writes sel / sel_count), attend only (reads them) and
 // full (A-E in one launch, the selection never leaves the chip).
 #include <algorithm>
@@ -38,11 +44,15 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kStageRows = 256;                    // code rows per bulk stage
+constexpr int kStageRows = 256;                      // code rows per bulk stage
 constexpr int kStages = 2;
 constexpr int kStageBytes = kStageRows * kRowBytes;  // 16 KiB
-constexpr int kPagesPerRound = kWarps;             // one page per warp
-constexpr int kPageSmem = 4 * 2048;                // K lo/hi, V lo/hi halves
+constexpr int kPageSmem = 4 * 2048;                  // K lo/hi, V lo/hi halves
+constexpr int kMaxSlots = 2;                         // page buffers per warp
+constexpr int kBins = 1024;                          // value histogram
+constexpr int kMaxCand = 1024;                       // boundary-bin candidates
+constexpr int kMaxBitmapWords = (ABSP_MAX_BLOCKS_PER_HEAD + 31) / 32;
+constexpr int kSelectScratch = (kBins + 2 * kMaxCand + 2 * kMaxBitmapWords) * 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Params {
@@ -60,15 +70,20 @@ struct Params {
     float qk_scale_log2;          // log2(e) / sqrt(128)
     uint32_t regA_off;            // byte offsets inside the aligned smem base
     uint32_t small_off;
+    uint32_t scratch_off;         // select scratch inside region B
+    int32_t slots;                // page buffers per warp (1 or 2)
 };
 
 struct Small {                    // fixed-size shared scratch
-    unsigned long long bar[4];    // code stage 0/1, attention, spare
-    uint32_t hist[256];
-    int32_t misc[32];
+    unsigned long long bar_code[kStages];
+    unsigned long long bar_page[kWarps][kMaxSlots];
+    unsigned long long bar_merge;
+    unsigned long long bar_score;
+    float2 cmm[16];               // (min, max) of each cluster CTA's scores
+    int32_t misc[16];
+    float red[2][kWarps];
     float w[kD];                  // qbar[ch] * scale[ch]
     float zb[kD];                 // 2^23 + zp[ch]
-    int4 pinfo[kPagesPerRound];   // {phys, valid, -, -}
     uint32_t scan[kWarps];
 };
 
@@ -77,11 +92,17 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Monotone (non-decreasing) map of a score onto kBins bins of [mn, mx].
+__device__ __forceinline__ int value_bin(float x, float mn, float inv) {
+    return __float2int_rz(fminf((x - mn) * inv, static_cast<float>(kBins - 1)));
+}
+
 __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
     return *reinterpret_cast<const uint32_t*>(p);
 }
 
-// Block-wide exclusive prefix sum of one uint32 per thread.
+// Block-wide exclusive prefix sum of one uint32 per thread (one barrier;
+// `scan` must not be rewritten before the next barrier).
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* scan) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t inc = v;
@@ -92,57 +113,51 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* scan) 
     }
     if (lane == 31) scan[warp] = inc;
     __syncthreads();
+    const uint4 a = reinterpret_cast<const uint4*>(scan)[0];
+    const uint4 b = reinterpret_cast<const uint4*>(scan)[1];
+    const uint32_t t[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     uint32_t base = 0;
-    for (int w = 0; w < warp; ++w) base += scan[w];
-    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) base += w < warp ? t[w] : 0u;
     return base + inc - v;
 }
 
-// Top-k of keys[0..n) (largest keys, ties to the lower index), written to
-// out[0..k) in ascending index order.  Requires n <= 65535.
-__device__ void block_topk(const uint32_t* keys, int n, int k, int32_t* out, Small& sm) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (k >= n) {
-        for (int i = tid; i < n; i += kThreads) out[i] = i;
-        __syncthreads();
-        return;
+// Warp-wide exclusive prefix sum.
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v) {
+    const int lane = threadIdx.x & 31;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
     }
+    return inc - v;
+}
+
+// Threshold of the top-k by 4 passes of 8-bit radix select over the
+// order-preserving keys (keys > T are in, plus `rem` keys equal to T).
+__device__ __forceinline__ void radix_threshold(const float* sc, int n, int k, uint32_t* hist, Small& sm,
+                                uint32_t* T_out, int* rem_out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t prefix = 0, mask = 0;
     int rem = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
-        sm.hist[tid] = 0;  // kThreads == 256 bins
+        hist[tid] = 0;  // kThreads == 256 digits
         __syncthreads();
         for (int i = tid; i < n; i += kThreads) {
-            const uint32_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 0xFFu], 1u);
+            const uint32_t key = order_key(sc[i]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
         }
         __syncthreads();
-        if (warp == 0) {
-            // lane l scans digits 255-8l down to 248-8l
-            uint32_t c[8], tot = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                c[j] = sm.hist[255 - 8 * lane - j];
-                tot += c[j];
-            }
-            uint32_t inc = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += t;
-            }
-            const uint32_t exc = inc - tot;
-            if (exc < static_cast<uint32_t>(rem) && static_cast<uint32_t>(rem) <= inc) {
-                uint32_t cum = exc;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (cum + c[j] >= static_cast<uint32_t>(rem)) {
-                        sm.misc[0] = 255 - 8 * lane - j;
-                        sm.misc[1] = rem - static_cast<int>(cum);
-                        break;
-                    }
-                    cum += c[j];
-                }
+        {
+            // thread t owns digit 255 - t: an exclusive scan in thread order
+            // counts the candidates with a larger digit
+            const int dgt = 255 - tid;
+            const uint32_t c = hist[dgt];
+            const uint32_t above = block_excl_scan(c, sm.scan);
+            if (above < static_cast<uint32_t>(rem) && static_cast<uint32_t>(rem) <= above + c) {
+                sm.misc[0] = dgt;
+                sm.misc[1] = rem - static_cast<int>(above);
             }
         }
         __syncthreads();
@@ -151,39 +166,189 @@ __device__ void block_topk(const uint32_t* keys, int n, int k, int32_t* out, Sma
         rem = sm.misc[1];
         __syncthreads();
     }
-    // keys > T are in; of the keys == T the `rem` lowest indices are in.
-    const uint32_t T = prefix;
-    const int per = (n + kThreads - 1) / kThreads;
-    const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+    *T_out = prefix;
+    *rem_out = rem;
+}
+
+// Ordered compaction of the top-k by a threshold: keys > T are in, and of
+// the keys == T the `rem` lowest indices.  Each warp compacts a contiguous
+// index range 32 scores at a time with ballots.
+__device__ __forceinline__ void compact_by_threshold(const float* sc, int n, uint32_t T, int rem, int32_t* out,
+                                     Small& sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per_w = (n + kWarps - 1) / kWarps;
+    const int w0 = min(n, warp * per_w), w1 = min(n, w0 + per_w);
     uint32_t gt = 0, eq = 0;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t key = keys[i];
-        gt += key > T;
-        eq += key == T;
+    for (int b = w0; b < w1; b += 32) {
+        const int i = b + lane;
+        const uint32_t key = i < w1 ? order_key(sc[i]) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, i < w1 && key > T));
+        eq += __popc(__ballot_sync(0xffffffffu, i < w1 && key == T));
     }
-    const uint32_t ex = block_excl_scan((gt << 16) | eq, sm.scan);
+    if (lane == 0) sm.scan[warp] = (gt << 16) | eq;
+    __syncthreads();
+    uint32_t ex = 0;
+    for (int w = 0; w < warp; ++w) ex += sm.scan[w];
     uint32_t gtb = ex >> 16, eqb = ex & 0xFFFFu;
     const uint32_t r = static_cast<uint32_t>(rem);
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t key = keys[i];
-        if (key > T) {
-            out[gtb + min(eqb, r)] = i;
-            ++gtb;
-        } else if (key == T) {
-            if (eqb < r) out[gtb + eqb] = i;
-            ++eqb;
-        }
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int b = w0; b < w1; b += 32) {
+        const int i = b + lane;
+        const uint32_t key = i < w1 ? order_key(sc[i]) : 0u;
+        const bool isg = i < w1 && key > T, ise = i < w1 && key == T;
+        const uint32_t bg = __ballot_sync(0xffffffffu, isg);
+        const uint32_t be = __ballot_sync(0xffffffffu, ise);
+        const uint32_t gp = gtb + __popc(bg & lt), ep = eqb + __popc(be & lt);
+        if (isg) out[gp + min(ep, r)] = i;
+        else if (ise && ep < r) out[gp + ep] = i;
+        gtb += __popc(bg);
+        eqb += __popc(be);
     }
     __syncthreads();
 }
 
-template <int MODE, bool BIG_GROUP>
+// Ascending list of the set bits of bitmap[0..nwords), by one warp.
+__device__ __forceinline__ void warp_compact_bitmap(const uint32_t* bitmap, int nwords,
+                                                    int32_t* out) {
+    const int lane = threadIdx.x & 31;
+    const int wpl = (nwords + 31) / 32;
+    const int j0 = min(nwords, lane * wpl), j1 = min(nwords, j0 + wpl);
+    uint32_t cnt = 0;
+    for (int j = j0; j < j1; ++j) cnt += __popc(bitmap[j]);
+    uint32_t pos = warp_excl_scan(cnt);
+    for (int j = j0; j < j1; ++j) {
+        uint32_t bits = bitmap[j];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            out[pos++] = j * 32 + b;
+            bits &= bits - 1u;
+        }
+    }
+}
+
+// Top-k of sc[0..n) (largest scores, ties to the lower index), written to
+// out[0..k) in ascending index order; [mn, mx] is the range of the scores.
+// The kBins histogram bins at the start of `scratch` must be zero on entry.
+// n <= 65535.
+__device__ __forceinline__ void block_topk(const float* sc, int n, int k, float mn, float mx, int32_t* out,
+                           uint32_t* scratch, Small& sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (k >= n) {
+        for (int i = tid; i < n; i += kThreads) out[i] = i;
+        __syncthreads();
+        return;
+    }
+    uint32_t* hist = scratch;
+    uint32_t* ckey = scratch + kBins;
+    int32_t* cidx = reinterpret_cast<int32_t*>(scratch + kBins + kMaxCand);
+    uint32_t* bitmap = scratch + kBins + 2 * kMaxCand;
+    const float inv = static_cast<float>(kBins) / (mx - mn);
+    if (!(mx > mn)) {                 // every score equal: lowest k indices
+        compact_by_threshold(sc, n, order_key(mx), k, out, sm);
+        return;
+    }
+    if (inv < INFINITY) {
+        // histogram of the scores over kBins equal bins of [mn, mx]; the
+        // bins were zeroed by the caller
+        constexpr int U = 8;
+        for (int b = tid; b < n; b += kThreads * U) {
+            float x[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) x[u] = b + u * kThreads < n ? sc[b + u * kThreads] : mn;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (b + u * kThreads < n) atomicAdd(&hist[value_bin(x[u], mn, inv)], 1u);
+        }
+        __syncthreads();
+        {
+            // thread t owns bins 4(255-t) .. 4(255-t)+3 (one 16-byte load);
+            // an exclusive scan in thread order counts the scores above them
+            const uint4 hv = reinterpret_cast<const uint4*>(hist)[255 - tid];
+            const uint32_t tot = hv.x + hv.y + hv.z + hv.w;
+            const uint32_t above = block_excl_scan(tot, sm.scan);
+            if (above < static_cast<uint32_t>(k) && static_cast<uint32_t>(k) <= above + tot) {
+                const uint32_t c[4] = {hv.w, hv.z, hv.y, hv.x};  // descending bins
+                uint32_t cum = above;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (cum < static_cast<uint32_t>(k) && static_cast<uint32_t>(k) <= cum + c[j]) {
+                        sm.misc[0] = 4 * (255 - tid) + 3 - j;
+                        sm.misc[1] = k - static_cast<int>(cum);
+                        sm.misc[2] = static_cast<int>(c[j]);
+                    }
+                    cum += c[j];
+                }
+            }
+        }
+        __syncthreads();
+        const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
+        if (m <= kMaxCand) {
+            // one pass: per 32 scores, a ballot word of the scores above bin
+            // bstar (in) and one of the scores inside it (candidates)
+            uint32_t* inw = bitmap;
+            uint32_t* eqw = bitmap + kMaxBitmapWords;
+            const int nwords = (n + 31) / 32;
+            constexpr int V = 8;
+            for (int w0 = warp; w0 < nwords; w0 += kWarps * V) {
+                float x[V];
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    const int i = (w0 + v * kWarps) * 32 + lane;
+                    x[v] = (w0 + v * kWarps < nwords && i < n) ? sc[i] : mn;
+                }
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    const int wd = w0 + v * kWarps;
+                    const bool live = wd < nwords && wd * 32 + lane < n;
+                    const int bn = value_bin(x[v], mn, inv);
+                    const uint32_t gw = __ballot_sync(0xffffffffu, live && bn > bstar);
+                    const uint32_t ew = __ballot_sync(0xffffffffu, live && bn == bstar);
+                    if (lane == 0 && wd < nwords) {
+                        inw[wd] = gw;
+                        eqw[wd] = ew;
+                    }
+                }
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // warp 0: list the candidates, rank them exactly (ties to the
+                // lower index), add the `need` best to the bitmap, compact
+                warp_compact_bitmap(eqw, nwords, cidx);
+                __syncwarp();
+                for (int c = lane; c < m; c += 32) ckey[c] = order_key(sc[cidx[c]]);
+                __syncwarp();
+                for (int c = lane; c < m; c += 32) {
+                    const uint32_t key = ckey[c];
+                    const int idx = cidx[c];
+                    int rank = 0;
+                    for (int j = 0; j < m; ++j) {
+                        const uint32_t kj = ckey[j];
+                        rank += (kj > key) || (kj == key && j < c);   // cidx ascending
+                    }
+                    if (rank < need) atomicOr(&inw[idx >> 5], 1u << (idx & 31));
+                }
+                __syncwarp();
+                warp_compact_bitmap(inw, nwords, out);
+            }
+            __syncthreads();
+            return;
+        }
+        __syncthreads();
+    }
+    uint32_t T = 0;
+    int rem = 0;
+    radix_threshold(sc, n, k, scratch, sm, &T, &rem);
+    compact_by_threshold(sc, n, T, rem, out, sm);
+}
+
+template <int MODE, bool BIG_GROUP, bool EARLY>
 __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base, derived from the shared array by a byte offset
+    // so that every access below stays in the shared address space
+    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* regB = base;                        // scores / pages / warp merge
     uint8_t* regA = base + p.regA_off;           // code ring / cluster merge
     Small& sm = *reinterpret_cast<Small*>(base + p.small_off);
@@ -195,56 +360,83 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
     const int pair = blockIdx.x / C;
     const int Hkv = p.kv.Hkv, G = p.kv.G;
     const int s = pair / Hkv, h = pair % Hkv;
-    const uint32_t bar_code0 = smem_u32(&sm.bar[0]);
-    const uint32_t bar_attn = smem_u32(&sm.bar[2]);
+    const int NB = p.slots;
+    const int bs = p.kv.bs[h];
+    const int spb = bs / kPage;
+    const int32_t* pt = p.kv.page_table + static_cast<int64_t>(s) * p.kv.max_pages;
+    constexpr bool kSelect = (MODE & kModeSelect) != 0;
+    constexpr bool kAttend = (MODE & kModeAttend) != 0;
 
-    // B0 arrive: matched by the wait before the first remote access.
-    cluster_arrive_relaxed();
     if (tid == 0) {
-        mbar_init(bar_code0, 1);
-        mbar_init(bar_code0 + 8, 1);
-        mbar_init(bar_attn, 1);
+        for (int i = 0; i < kStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
+        for (int w = 0; w < kWarps; ++w)
+            for (int i = 0; i < kMaxSlots; ++i) mbar_init(smem_u32(&sm.bar_page[w][i]), 1);
+        mbar_init(smem_u32(&sm.bar_score), 1);
+        if (C > 1) mbar_init(smem_u32(&sm.bar_merge), C - 1);
         fence_mbar_init();
     }
-    // Nothing in global memory is read before this point.
-    pdl_wait();
-    pdl_trigger();
-    __syncthreads();
-
+    // Without EARLY nothing in global memory is read before this wait.
+    if constexpr (!EARLY) {
+        pdl_wait();
+        pdl_trigger();
+    }
     int len = p.kv.seq_lens[s];
     if (len < 0 || len > p.kv.max_pages * kPage) {
         if (tid == 0 && rank == 0 && h == 0) set_error(p.err, ABSP_ERR_DEVICE_FAULT, s);
         len = 0;
     }
-    const int bs = p.kv.bs[h];
-    const int spb = bs / kPage;
     const int n = (len + bs - 1) / bs;
-    int K = 0;
-
-    if constexpr ((MODE & kModeSelect) != 0) {
-        // ---------------------------------------------------- A: score --
-        K = min(n, max(1, p.budget / bs));
-        const int per = (n + static_cast<int>(C) - 1) / static_cast<int>(C);
-        const int r0 = min(n, static_cast<int>(rank) * per);
-        const int nrows = min(n, r0 + per) - r0;
-        const int nchunks = (nrows + kStageRows - 1) / kStageRows;
-        const uint8_t* cbase =
-            p.codes + (static_cast<int64_t>(s) * p.kv.rows_per_seq + p.kv.row_base[h] + r0) * kRowBytes;
-        if (tid == 0) {
+    // rows of this CTA: a contiguous range, a multiple of 4 rows long
+    const int per = ((n + static_cast<int>(C) - 1) / static_cast<int>(C) + 3) & ~3;
+    const int r0 = min(n, static_cast<int>(rank) * per);
+    const int nrows = min(n, r0 + per) - r0;
+    const int nchunks = (nrows + kStageRows - 1) / kStageRows;
+    const uint8_t* cbase =
+        p.codes + (static_cast<int64_t>(s) * p.kv.rows_per_seq + p.kv.row_base[h] + r0) * kRowBytes;
+    if (tid == 0) {
+        if (kSelect && (MODE != kModeSelect || rank == 0))
+            mbar_arrive_expect_tx(smem_u32(&sm.bar_score), 16 * ((n + 3) / 4) + 8 * C);
+        if (kSelect) {
             for (int c = 0; c < min(nchunks, kStages); ++c) {
                 const int rows = min(kStageRows, nrows - c * kStageRows);
-                mbar_arrive_expect_tx(bar_code0 + 8 * c, rows * kRowBytes);
+                const uint32_t bar = smem_u32(&sm.bar_code[c]);
+                mbar_arrive_expect_tx(bar, rows * kRowBytes);
                 bulk_g2s(smem_u32(regA + c * kStageBytes), cbase + c * kStageBytes,
-                         rows * kRowBytes, bar_code0 + 8 * c);
+                         rows * kRowBytes, bar);
             }
         }
+    }
+    // B0 arrive (release: the barrier set-up above is visible cluster-wide
+    // once B0 completes); matched by the wait before the first remote access.
+    cluster_arrive();
+    if constexpr (kAttend) {
+        // the attention phase reads page-table entries of this sequence
+        const int npg = (len + kPage - 1) / kPage;
+        for (int i = tid * 32; i < npg; i += kThreads * 32) prefetch_l2(pt + i);
+    }
+    float scl = 0.0f;
+    int32_t zpv = 0;
+    if (kSelect && tid < kD) {
+        const int64_t pi = (static_cast<int64_t>(s) * Hkv + h) * kD + tid;
+        scl = p.scale[pi];
+        zpv = p.zp[pi];
+    }
+    if constexpr (EARLY) {
+        // only the query may be produced by the preceding kernel
+        pdl_wait();
+        pdl_trigger();
+    }
+    int K = 0;
+
+    if constexpr (kSelect) {
+        // ---------------------------------------------------- A: score --
+        K = min(n, max(1, p.budget / bs));
         if (tid < kD) {
             const __nv_bfloat16* qh = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD + tid;
             float qb = 0.0f;
             for (int j = 0; j < G; ++j) qb += __bfloat162float(qh[j * kD]);
-            const int64_t pi = (static_cast<int64_t>(s) * Hkv + h) * kD + tid;
-            sm.w[tid] = qb * p.scale[pi];
-            sm.zb[tid] = 8388608.0f + static_cast<float>(p.zp[pi]);
+            sm.w[tid] = qb * scl;
+            sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
         }
         __syncthreads();
         const int sub = tid & 7, grp = tid >> 3;  // 32 groups of 8 lanes
@@ -256,58 +448,107 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         }
         float* scores = reinterpret_cast<float*>(regB);
         const uint32_t scores_u32 = smem_u32(scores);
+        const uint32_t bar_score = smem_u32(&sm.bar_score);
+        float lmin = INFINITY, lmax = -INFINITY;
         cluster_wait();  // B0: every CTA of the cluster is running
+        {   // histogram bins of the select, zeroed while the codes stream in
+            uint32_t* hist = reinterpret_cast<uint32_t*>(regB + p.scratch_off);
+            for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+        }
         for (int c = 0; c < nchunks; ++c) {
             const int stage = c % kStages;
-            mbar_wait_bounded(bar_code0 + 8 * stage, (c / kStages) & 1, p.err, 1);
+            mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / kStages) & 1, p.err, 1);
             const int rows = min(kStageRows, nrows - c * kStageRows);
             const uint8_t* sbuf = regA + stage * kStageBytes;
-            for (int rb = 0; rb < rows; rb += kThreads / 8) {
-                const int r = rb + grp;
-                const bool ok = r < rows;
-                uint2 x = make_uint2(0u, 0u);
-                if (ok) x = *reinterpret_cast<const uint2*>(sbuf + r * kRowBytes + sub * 8);
-                float acc = 0.0f;
+            // each 8-lane group scores 4 consecutive rows
+            for (int rb = 0; rb < rows; rb += 4 * (kThreads / 8)) {
+                const int r4 = rb + 4 * grp;
+                float q4[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float f = __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
-                    acc = fmaf(wr[k], f, acc);
-                }
+                for (int u = 0; u < 4; ++u) {
+                    const int r = r4 + u;
+                    uint2 x = make_uint2(0u, 0u);
+                    if (r < rows) x = *reinterpret_cast<const uint2*>(sbuf + r * kRowBytes + sub * 8);
+                    float acc = 0.0f;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float f =
-                        __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
-                    acc = fmaf(wr[8 + k], f, acc);
+                    for (int k = 0; k < 8; ++k) {
+                        const float f =
+                            __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
+                        acc = fmaf(wr[k], f, acc);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float f =
+                            __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
+                        acc = fmaf(wr[8 + k], f, acc);
+                    }
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                    q4[u] = r < rows ? acc : 0.0f;
+                    if (r < rows) {
+                        lmin = fminf(lmin, acc);
+                        lmax = fmaxf(lmax, acc);
+                    }
                 }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                if (ok) {
-                    const uint32_t row = static_cast<uint32_t>(r0 + c * kStageRows + r);
-                    for (uint32_t dst = sub; dst < C; dst += 8)
-                        dsmem_st_f32(dsmem_addr(scores_u32 + 4 * row, dst), acc);
+                if (r4 < rows) {
+                    const uint32_t off = 4u * static_cast<uint32_t>(r0 + c * kStageRows + r4);
+                    if (MODE == kModeSelect) {
+                        if (sub == 0)
+                            st_async_v4(dsmem_addr(scores_u32 + off, 0), q4[0], q4[1], q4[2],
+                                        q4[3], dsmem_addr(bar_score, 0));
+                    } else {
+                        for (uint32_t dst = sub; dst < C; dst += 8)
+                            st_async_v4(dsmem_addr(scores_u32 + off, dst), q4[0], q4[1], q4[2],
+                                        q4[3], dsmem_addr(bar_score, dst));
+                    }
                 }
             }
             __syncthreads();
             if (tid == 0 && c + kStages < nchunks) {
                 const int cn = c + kStages;
                 const int rows_n = min(kStageRows, nrows - cn * kStageRows);
+                const uint32_t bar = smem_u32(&sm.bar_code[stage]);
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(bar_code0 + 8 * stage, rows_n * kRowBytes);
+                mbar_arrive_expect_tx(bar, rows_n * kRowBytes);
                 bulk_g2s(smem_u32(regA + stage * kStageBytes), cbase + cn * kStageBytes,
-                         rows_n * kRowBytes, bar_code0 + 8 * stage);
+                         rows_n * kRowBytes, bar);
             }
         }
-        // ---------------------------------------------- B: all scores in --
-        cluster_arrive();
-        cluster_wait();
-        if (MODE == kModeSelect && rank != 0) return;  // no remote access follows
+        // this CTA's score range, sent along with the scores
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
+            lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+        }
+        if (lane == 0) {
+            sm.red[0][warp] = lmin;
+            sm.red[1][warp] = lmax;
+        }
+        __syncthreads();
+        if (tid < static_cast<int>(C) && (MODE != kModeSelect || tid == 0)) {
+            float a = sm.red[0][0], b = sm.red[1][0];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) {
+                a = fminf(a, sm.red[0][w]);
+                b = fmaxf(b, sm.red[1][w]);
+            }
+            st_async_v2(dsmem_addr(smem_u32(&sm.cmm[rank]), tid), a, b,
+                        dsmem_addr(bar_score, tid));
+        }
+        // select-only: CTA 0 alone receives and selects
+        if (MODE == kModeSelect && rank != 0) return;
+        // ------------------------------------- B: every score arrived --
+        mbar_wait_bounded<true>(bar_score, 0, p.err, 4);
 
         // --------------------------------------------------- C: select --
-        uint32_t* keys = reinterpret_cast<uint32_t*>(regB);
-        for (int i = tid; i < n; i += kThreads) keys[i] = order_key(scores[i]);
-        __syncthreads();
-        block_topk(keys, n, K, sel_s, sm);
+        float smin = INFINITY, smax = -INFINITY;
+        for (uint32_t r = 0; r < C; ++r) {
+            smin = fminf(smin, sm.cmm[r].x);
+            smax = fmaxf(smax, sm.cmm[r].y);
+        }
+        block_topk(scores, n, K, smin, smax, sel_s,
+                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm);
         if (MODE == kModeSelect) {
             int32_t* dst = p.sel + (static_cast<int64_t>(s) * Hkv + h) * p.kmax;
             for (int i = tid; i < K; i += kThreads) dst[i] = sel_s[i];
@@ -338,6 +579,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         const int P = K * spb;
         const int pb = static_cast<int>((static_cast<int64_t>(P) * rank) / C);
         const int pe = static_cast<int>((static_cast<int64_t>(P) * (rank + 1)) / C);
+        const int cnt_w = pe - pb > warp ? (pe - pb - warp + kWarps - 1) / kWarps : 0;
         const int g = lane >> 2, t4 = lane & 3;
         const __nv_bfloat16* qg = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
         uint32_t qa0[8], qa2[8], qa1[8], qa3[8];
@@ -358,17 +600,16 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
         float m0 = -FLT_MAX, m8 = -FLT_MAX, l0 = 0.0f, l8 = 0.0f;
         bool any0 = false;  // this warp has seen at least one valid token
-        const int32_t* pt = p.kv.page_table + static_cast<int64_t>(s) * p.kv.max_pages;
         const float qks = p.qk_scale_log2;
-        __syncthreads();  // the score keys in regB are dead from here on
+        uint8_t* wbuf = regB + warp * NB * kPageSmem;  // this warp's page slots
 
-        int round = 0;
-        for (int bp = pb; bp < pe; bp += kPagesPerRound, ++round) {
-            const int np = min(kPagesPerRound, pe - bp);
-            if (tid < np) {
-                const int j = bp + tid;
+        // page i of this warp: selection entry, bounds checks, tensor copies
+        auto issue = [&](int i) -> int {
+            int valid = 0;
+            if (lane == 0) {
+                const int j = pb + warp + kWarps * i;
                 const int b = sel_s[j / spb];
-                int valid = 0, phys = -1;
+                int phys = -1;
                 if (b >= 0) {
                     const int lp = b * spb + (j % spb);
                     valid = min(kPage, len - lp * kPage);
@@ -382,28 +623,32 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
                         valid = 0;
                     }
                 }
-                sm.pinfo[tid] = make_int4(phys, valid, 0, 0);
-            }
-            __syncthreads();
-            if (tid == 0) {
-                uint32_t bytes = 0;
-                for (int i = 0; i < np; ++i) bytes += sm.pinfo[i].y > 0 ? kPageSmem : 0;
+                const int slot = i % NB;
+                const uint32_t bar = smem_u32(&sm.bar_page[warp][slot]);
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(bar_attn, bytes);
-                for (int i = 0; i < np; ++i) {
-                    if (sm.pinfo[i].y <= 0) continue;
-                    const int y = (sm.pinfo[i].x * Hkv + h) * kPage;
-                    const uint32_t dst = smem_u32(regB + i * kPageSmem);
-                    tma_load_2d(dst, &tmk, 0, y, bar_attn);
-                    tma_load_2d(dst + 2048, &tmk, 64, y, bar_attn);
-                    tma_load_2d(dst + 4096, &tmv, 0, y, bar_attn);
-                    tma_load_2d(dst + 6144, &tmv, 64, y, bar_attn);
+                mbar_arrive_expect_tx(bar, valid > 0 ? kPageSmem : 0);
+                if (valid > 0) {
+                    const int y = (phys * Hkv + h) * kPage;
+                    const uint32_t dst = smem_u32(wbuf + slot * kPageSmem);
+                    tma_load_2d(dst, &tmk, 0, y, bar);
+                    tma_load_2d(dst + 2048, &tmk, 64, y, bar);
+                    tma_load_2d(dst + 4096, &tmv, 0, y, bar);
+                    tma_load_2d(dst + 6144, &tmv, 64, y, bar);
                 }
             }
-            mbar_wait_bounded(bar_attn, round & 1, p.err, 2);
-            const int valid = warp < np ? sm.pinfo[warp].y : 0;
+            return __shfl_sync(0xffffffffu, valid, 0);
+        };
+
+        __syncthreads();  // every thread is done with the scores in region B
+        int vq0 = 0, vq1 = 0;
+        if (cnt_w > 0) vq0 = issue(0);
+        if (NB > 1 && cnt_w > 1) vq1 = issue(1);
+        for (int i = 0; i < cnt_w; ++i) {
+            const int slot = i % NB;
+            const int valid = slot == 0 ? vq0 : vq1;
+            mbar_wait_bounded(smem_u32(&sm.bar_page[warp][slot]), (i / NB) & 1, p.err, 2);
             if (valid > 0) {
-                uint8_t* pg = regB + warp * kPageSmem;
+                uint8_t* pg = wbuf + slot * kPageSmem;
                 const uint32_t kb = smem_u32(pg), vb = kb + 4096;
                 if (valid < kPage) {
                     // zero the V rows past the sequence end (they may hold
@@ -437,10 +682,10 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
                 }
                 // scale to log2 units and mask tokens past the end
                 const int ta = 2 * t4, tb = 8 + 2 * t4;
-                float x0 = ta < valid ? s0[0] * qks : -INFINITY;
-                float x1 = ta + 1 < valid ? s0[1] * qks : -INFINITY;
-                float x2 = tb < valid ? s1[0] * qks : -INFINITY;
-                float x3 = tb + 1 < valid ? s1[1] * qks : -INFINITY;
+                const float x0 = ta < valid ? s0[0] * qks : -INFINITY;
+                const float x1 = ta + 1 < valid ? s0[1] * qks : -INFINITY;
+                const float x2 = tb < valid ? s1[0] * qks : -INFINITY;
+                const float x3 = tb + 1 < valid ? s1[1] * qks : -INFINITY;
                 float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -449,16 +694,15 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
                 const float corr0 = any0 ? exp2f(m0 - mn0) : 0.0f;
                 const uint32_t pa0 = pack_bf16x2(exp2f(x0 - mn0), exp2f(x1 - mn0));
                 const uint32_t pa2 = pack_bf16x2(exp2f(x2 - mn0), exp2f(x3 - mn0));
-                const float ps0 = bf16lo(pa0) + bf16hi(pa0) + bf16lo(pa2) + bf16hi(pa2);
-                l0 = l0 * corr0 + ps0;
+                l0 = l0 * corr0 + (bf16lo(pa0) + bf16hi(pa0) + bf16lo(pa2) + bf16hi(pa2));
                 m0 = mn0;
                 uint32_t pa1 = 0u, pa3 = 0u;
                 float corr8 = 1.0f;
                 if constexpr (BIG_GROUP) {
-                    float y0 = ta < valid ? s0[2] * qks : -INFINITY;
-                    float y1 = ta + 1 < valid ? s0[3] * qks : -INFINITY;
-                    float y2 = tb < valid ? s1[2] * qks : -INFINITY;
-                    float y3 = tb + 1 < valid ? s1[3] * qks : -INFINITY;
+                    const float y0 = ta < valid ? s0[2] * qks : -INFINITY;
+                    const float y1 = ta + 1 < valid ? s0[3] * qks : -INFINITY;
+                    const float y2 = tb < valid ? s1[2] * qks : -INFINITY;
+                    const float y3 = tb + 1 < valid ? s1[3] * qks : -INFINITY;
                     float my = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
                     my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, 1));
                     my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, 2));
@@ -466,17 +710,17 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
                     corr8 = any0 ? exp2f(m8 - mn8) : 0.0f;
                     pa1 = pack_bf16x2(exp2f(y0 - mn8), exp2f(y1 - mn8));
                     pa3 = pack_bf16x2(exp2f(y2 - mn8), exp2f(y3 - mn8));
-                    l8 = l8 * corr8 + bf16lo(pa1) + bf16hi(pa1) + bf16lo(pa3) + bf16hi(pa3);
+                    l8 = l8 * corr8 + (bf16lo(pa1) + bf16hi(pa1) + bf16lo(pa3) + bf16hi(pa3));
                     m8 = mn8;
                 }
                 any0 = true;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    o[i][0] *= corr0;
-                    o[i][1] *= corr0;
+                for (int t = 0; t < 16; ++t) {
+                    o[t][0] *= corr0;
+                    o[t][1] *= corr0;
                     if constexpr (BIG_GROUP) {
-                        o[i][2] *= corr8;
-                        o[i][3] *= corr8;
+                        o[t][2] *= corr8;
+                        o[t][3] *= corr8;
                     }
                 }
                 // O[row][d] += P[row][token] V[token][d]
@@ -498,7 +742,12 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
                     }
                 }
             }
-            __syncthreads();  // page buffers are reused next round
+            fence_proxy_async_smem();  // this lane's reads/writes of the slot
+            __syncwarp();              // before the slot's next tensor copy
+            if (i + NB < cnt_w) {
+                const int v = issue(i + NB);
+                if (slot == 0) vq0 = v; else vq1 = v;
+            }
         }
         l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
         l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -510,14 +759,15 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         }
 
         // ------------------------------------------- E: merge partials --
-        float* Ow = reinterpret_cast<float*>(regB);       // [warps][G][128]
+        __syncthreads();                                   // page slots are dead
+        float* Ow = reinterpret_cast<float*>(regB);        // [warps][G][128]
         float* mw = Ow + kWarps * G * kD;                  // [warps][G]
         float* lw = mw + kWarps * G;
         if (g < G) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                Ow[(warp * G + g) * kD + i * 8 + 2 * t4] = o[i][0];
-                Ow[(warp * G + g) * kD + i * 8 + 2 * t4 + 1] = o[i][1];
+            for (int t = 0; t < 16; ++t) {
+                Ow[(warp * G + g) * kD + t * 8 + 2 * t4] = o[t][0];
+                Ow[(warp * G + g) * kD + t * 8 + 2 * t4 + 1] = o[t][1];
             }
             if (t4 == 0) {
                 mw[warp * G + g] = m0;
@@ -527,9 +777,9 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         if constexpr (BIG_GROUP) {
             if (g + 8 < G) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    Ow[(warp * G + g + 8) * kD + i * 8 + 2 * t4] = o[i][2];
-                    Ow[(warp * G + g + 8) * kD + i * 8 + 2 * t4 + 1] = o[i][3];
+                for (int t = 0; t < 16; ++t) {
+                    Ow[(warp * G + g + 8) * kD + t * 8 + 2 * t4] = o[t][2];
+                    Ow[(warp * G + g + 8) * kD + t * 8 + 2 * t4 + 1] = o[t][3];
                 }
                 if (t4 == 0) {
                     mw[warp * G + g + 8] = m8;
@@ -557,6 +807,12 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
             }
             if (C == 1) {
                 outp[row * kD + d] = __float2bfloat16_rn(L > 0.0f ? Oacc / L : 0.0f);
+            } else if (rank == 0) {
+                partO[row * kD + d] = Oacc;
+                if (d == 0) {
+                    partM[row] = M;
+                    partL[row] = L;
+                }
             } else {
                 const uint32_t lo = smem_u32(&partO[(rank * G + row) * kD + d]);
                 dsmem_st_f32(dsmem_addr(lo, 0), Oacc);
@@ -567,33 +823,36 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
             }
         }
         if (C > 1) {
-            cluster_arrive();
-            cluster_wait();
-            if (rank == 0) {
-                for (int idx = tid; idx < G * kD; idx += kThreads) {
-                    const int row = idx >> 7, d = idx & (kD - 1);
-                    float M = -INFINITY;
-                    for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, partM[r * G + row]);
-                    float L = 0.0f, Oacc = 0.0f;
-                    if (M != -INFINITY) {
-                        for (uint32_t r = 0; r < C; ++r) {
-                            const float f = exp2f(partM[r * G + row] - M);
-                            L += partL[r * G + row] * f;
-                            Oacc += partO[(r * G + row) * kD + d] * f;
-                        }
+            __syncthreads();
+            if (rank != 0) {
+                // every partial of this CTA is written; tell CTA 0 and leave
+                if (tid == 0) mbar_arrive_remote(dsmem_addr(smem_u32(&sm.bar_merge), 0));
+                return;
+            }
+            mbar_wait_bounded<true>(smem_u32(&sm.bar_merge), 0, p.err, 3);
+            for (int idx = tid; idx < G * kD; idx += kThreads) {
+                const int row = idx >> 7, d = idx & (kD - 1);
+                float M = -INFINITY;
+                for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, partM[r * G + row]);
+                float L = 0.0f, Oacc = 0.0f;
+                if (M != -INFINITY) {
+                    for (uint32_t r = 0; r < C; ++r) {
+                        const float f = exp2f(partM[r * G + row] - M);
+                        L += partL[r * G + row] * f;
+                        Oacc += partO[(r * G + row) * kD + d] * f;
                     }
-                    outp[row * kD + d] = __float2bfloat16_rn(L > 0.0f ? Oacc / L : 0.0f);
                 }
+                outp[row * kD + d] = __float2bfloat16_rn(L > 0.0f ? Oacc / L : 0.0f);
             }
         }
     }
 }
 
-template <int MODE, bool BIG>
+template <int MODE, bool BIG, bool EARLY>
 cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool pdl,
                         const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st,
                         bool* fits) {
-    auto kern = decode_kernel<MODE, BIG>;
+    auto kern = decode_kernel<MODE, BIG, EARLY>;
     static bool configured = false;   // attributes are per function, set once
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -620,6 +879,7 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
     // can at least one cluster of this shape be resident?  (cached per shape)
     static int cache_c[8] = {0}, cache_fit[8] = {0};
     static size_t cache_smem[8] = {0};
+    static int next = 0;
     int fit = -1;
     for (int i = 0; i < 8; ++i)
         if (cache_c[i] == C && cache_smem[i] == smem) fit = cache_fit[i];
@@ -631,7 +891,6 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
             nclusters = 0;
         }
         fit = nclusters > 0 ? 1 : 0;
-        static int next = 0;
         cache_c[next] = C;
         cache_smem[next] = smem;
         cache_fit[next] = fit;
@@ -653,7 +912,7 @@ static int pick_cluster(int pairs, int num_sms) {
 }
 
 cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
-                          const CUtensorMap* tmv, bool pdl, cudaStream_t st) {
+                          const CUtensorMap* tmv, bool pdl, bool early_prefetch, cudaStream_t st) {
     static int num_sms = 0;
     if (num_sms == 0) {
         int dev = 0;
@@ -684,41 +943,58 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     int C = pick_cluster(pairs, num_sms);
     cudaError_t e = cudaSuccess;
     for (; C >= 1; C /= 2) {
-        size_t regB = 0, regA = 0;
+        // region B: scores + select scratch, or this CTA's page slots, or the
+        // warp merge; region A: code ring, or (CTA 0) the cluster merge
+        size_t regB = 0, regA = 0, scratch = 0;
+        int slots = 1;
         if (do_select) {
-            regB = std::max(regB, static_cast<size_t>(a.nmax) * 4);
+            // score slots for every row, rounded up to whole groups of 4
+            scratch = (static_cast<size_t>(a.nmax + 3) / 4) * 16;
+            regB = std::max(regB, scratch + kSelectScratch);
             regA = std::max(regA, static_cast<size_t>(kStages) * kStageBytes);
         }
         if (do_attend) {
-            regB = std::max(regB, static_cast<size_t>(kPagesPerRound) * kPageSmem);
+            const int pages_max = a.budget / kPage;         // pages selected per head
+            const int per_cta = (pages_max + C - 1) / C;
+            slots = per_cta > kWarps ? kMaxSlots : 1;
+            regB = std::max(regB, static_cast<size_t>(kWarps) * slots * kPageSmem);
             regB = std::max(regB, static_cast<size_t>(kWarps) * G * (kD + 2) * 4);
             if (C > 1) regA = std::max(regA, static_cast<size_t>(C) * G * (kD + 2) * 4);
         }
         regB = (regB + 1023) & ~static_cast<size_t>(1023);
         regA = (regA + 127) & ~static_cast<size_t>(127);
+        prm.scratch_off = static_cast<uint32_t>(scratch);
+        prm.slots = slots;
         prm.regA_off = static_cast<uint32_t>(regB);
         prm.small_off = static_cast<uint32_t>(regB + regA);
         const size_t smem = 1024 + regB + regA + sizeof(Small) + static_cast<size_t>(a.kmax) * 4;
         if (smem > 227 * 1024) return cudaErrorInvalidValue;
         bool fits = false;
-        switch (mode * 2 + (big ? 1 : 0)) {
-            case kModeSelect * 2:
-                e = launch_mode<kModeSelect, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+        const bool early = early_prefetch && mode == kModeFull;
+        switch (mode * 4 + (big ? 2 : 0) + (early ? 1 : 0)) {
+            case kModeSelect * 4:
+                e = launch_mode<kModeSelect, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
                 break;
-            case kModeSelect * 2 + 1:
-                e = launch_mode<kModeSelect, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+            case kModeSelect * 4 + 2:
+                e = launch_mode<kModeSelect, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
                 break;
-            case kModeAttend * 2:
-                e = launch_mode<kModeAttend, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+            case kModeAttend * 4:
+                e = launch_mode<kModeAttend, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
                 break;
-            case kModeAttend * 2 + 1:
-                e = launch_mode<kModeAttend, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+            case kModeAttend * 4 + 2:
+                e = launch_mode<kModeAttend, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
                 break;
-            case kModeFull * 2:
-                e = launch_mode<kModeFull, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+            case kModeFull * 4:
+                e = launch_mode<kModeFull, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+                break;
+            case kModeFull * 4 + 1:
+                e = launch_mode<kModeFull, false, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+                break;
+            case kModeFull * 4 + 2:
+                e = launch_mode<kModeFull, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
                 break;
             default:
-                e = launch_mode<kModeFull, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+                e = launch_mode<kModeFull, true, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
                 break;
         }
         if (e != cudaSuccess || fits) return e;

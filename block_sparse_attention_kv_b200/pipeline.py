@@ -51,9 +51,14 @@ class DeviceLayer:
                                self.sel_count, self.budget, self.out if out is None else out,
                                self.ws, self.stream)
 
-    def decode_step(self, q=None, out=None):
-        abi.absp_decode_step(self.kv, self.cent, self.data.q if q is None else q, self.budget,
-                             self.out if out is None else out, self.ws, self.stream)
+    def decode_step(self, q=None, out=None, flags: int = 0):
+        q = self.data.q if q is None else q
+        out = self.out if out is None else out
+        if flags:
+            abi.absp_decode_step_ex(self.kv, self.cent, q, self.budget, out, self.ws, flags,
+                                    self.stream)
+        else:
+            abi.absp_decode_step(self.kv, self.cent, q, self.budget, out, self.ws, self.stream)
 
     def decode_step_host(self, q_host, out_host):
         abi.absp_decode_step_host(self.kv, self.cent, q_host, self.budget, out_host, self.ws,

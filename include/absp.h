@@ -176,6 +176,25 @@ ABSP_API absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centro
                              const void* q, int32_t budget_tokens, void* out,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* Flags of absp_decode_step_ex. */
+#define ABSP_STEP_EARLY_PREFETCH 1u
+/* ABSP_STEP_EARLY_PREFETCH: the launch overlaps the tail of the preceding
+ * kernel in `stream` (programmatic dependent launch) and, before waiting for
+ * it, already reads the sequence lengths, page table, centroid codes and
+ * per-channel parameters; only the query is read after the wait.  The
+ * caller guarantees that the kernel issued immediately before this call in
+ * `stream` writes none of those buffers (it may write `q`).  This is the
+ * decode-loop case: the cache and centroids of a layer were written by
+ * earlier steps, the query by the kernel just before.  Without the flag
+ * nothing is read before the preceding kernel has completed. */
+
+/* absp_decode_step with flags (0 or ABSP_STEP_EARLY_PREFETCH); same
+ * results as absp_decode_step. */
+ABSP_API absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
+                                         const void* q, int32_t budget_tokens, void* out,
+                                         void* ws, size_t ws_bytes, uint32_t flags,
+                                         void* stream);
+
 /* absp_decode_step with HOST query and output buffers: copies q_host
  * (bf16 [S][Hq][128], pinned for true asynchrony) into the workspace, runs
  * the step and copies the result back to out_host, all on `stream`.  The

@@ -117,6 +117,13 @@ def test_small_workspace_rejected_before_launch(abi):
     assert e.value.status == abi.ABSP_ERR_INVALID_ARG
 
 
+def test_unknown_step_flags_rejected(abi):
+    kv = _kv(abi)
+    lib = abi.lib()
+    st = lib.absp_decode_step_ex(kv.ref, None, None, 1024, None, None, 0, 0x80, None)
+    assert st == abi.ABSP_ERR_INVALID_ARG
+
+
 def test_null_layer_and_status_strings(abi):
     lib = abi.lib()
     assert lib.absp_centroid_sizes(None, None, None, None) == abi.ABSP_ERR_INVALID_ARG

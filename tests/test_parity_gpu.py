@@ -48,6 +48,11 @@ def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None):
     dl.check()
     torch.cuda.synchronize()
     assert torch.equal(_bits(dl.out), _bits(out_split)), "fused step != select + decode"
+    dl.out.zero_()
+    dl.decode_step(flags=abi.ABSP_STEP_EARLY_PREFETCH)
+    dl.check()
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(dl.out), _bits(out_split)), "early-prefetch step differs"
 
     S, Hkv = d.num_seqs, d.num_kv_heads
     seqs = list(range(S)) if seqs is None else list(seqs)
@@ -144,6 +149,17 @@ def test_periodic_keys_resolve_ties_to_lower_index(lib):
             d.k_pages[ids, h] = k.view(256, 16, 128)
     rep, dl, res = run_case(lib, w, modify=modify)
     assert rep.near_ties == 0          # exact ties are resolved identically
+
+
+def test_outlier_block_forces_radix_fallback(lib):
+    # one block's keys scaled by 4096 stretch the score range so far that all
+    # other scores share one histogram bin: the select falls back to radix
+    w = synth.custom("outlier", 1, 8, 2, [32768], [16, 64], 1024, seed=32, planted_blocks=0)
+
+    def modify(d):
+        ids = d.page_table[0, 5:6].long()                 # block 5 of head 0 (bs 16)
+        d.k_pages[ids, 0] = (d.k_pages[ids, 0].float() * 4096.0).to(torch.bfloat16)
+    run_case(lib, w, modify=modify)
 
 
 def test_host_buffers_match_device_step(lib):
