@@ -7,10 +7,14 @@ drawn from {16, 32, 64} with probabilities {0.25, 0.25, 0.5}, token budget
 2048, INT4 centroids).  One benchmark step decodes one token through
 `--layers` (default 64) such layers, each with its own cache, centroids and
 query, so the working set (8 GiB) is far larger than L2.  Each layer-step is
-one absp_decode_step launch; the layer-steps of a step are captured in a
-CUDA graph and every launch waits for the previous one to finish before it
-reads anything (programmatic dependent launch only overlaps the launch
-latency), as consecutive layers of a real decode would.
+one absp_decode_step_ex launch with ABSP_STEP_EARLY_PREFETCH; the
+layer-steps of a step are captured in a CUDA graph.  Every launch waits for
+the previous one to finish before it reads its query, as consecutive layers
+of a real decode would; what overlaps the previous launch is only the
+launch itself and the reads of this layer's cache-side data (lengths, page
+table, centroid codes, per-channel parameters), which no decode kernel
+writes.  `variants.plain` is the same measurement with absp_decode_step
+(nothing read before the previous launch completed).
 
 value   = layer-steps/s over all ranks (weak scaling: every rank decodes its
           own layer stack, no collective on the data path);
@@ -172,6 +176,28 @@ def rebuild_bytes(d):
     return tot
 
 
+# ---------------------------------------------------------------- ranks --
+
+def rank_layer_ids(rank: int, layers: int) -> list:
+    """Layer seeds of one rank: every rank decodes its own layer stack."""
+    return [rank * layers + i for i in range(layers)]
+
+
+def reduce_max(value: float, dist=None, device=None) -> float:
+    """Max over ranks (identity on one process)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, layers: int, steps: int, ms: float) -> float:
+    """Whole-job layer-steps/s: all ranks' layer-steps over the max time."""
+    return world * layers * steps / (ms / 1e3)
+
+
 # ------------------------------------------------------- CPU oracle leg --
 
 def oracle_layer_sample(layer_index: int = 0):
@@ -271,8 +297,8 @@ def gpu_arm(args):
     stream = torch.cuda.Stream(device=dev)
     layers = []
     with torch.cuda.stream(stream):
-        for i in range(L):
-            d = synth.make_layer(w, rank * L + i, dev)
+        for i in rank_layer_ids(rank, L):
+            d = synth.make_layer(w, i, dev)
             layers.append(pipeline.DeviceLayer(d, stream=stream.cuda_stream))
     stream.synchronize()
 
@@ -310,8 +336,17 @@ def gpu_arm(args):
     bytes_per_launch = float(np.mean(nbytes))
 
     # CUDA graph of one step = L layer-steps
+    EARLY = abi.ABSP_STEP_EARLY_PREFETCH
+    for x in layers:                                   # warm the flagged variant
+        abi.absp_decode_step_ex(x.kv, x.cent, x.data.q, x.budget, x.out, x.ws, EARLY, sc)
+    stream.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
+        for x in layers:
+            abi.absp_decode_step_ex(x.kv, x.cent, x.data.q, x.budget, x.out, x.ws, EARLY, sc)
+    stream.synchronize()
+    g_plain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_plain, stream=stream):
         for x in layers:
             abi.absp_decode_step(x.kv, x.cent, x.data.q, x.budget, x.out, x.ws, sc)
     stream.synchronize()
@@ -332,20 +367,17 @@ def gpu_arm(args):
         torch.cuda.synchronize(dev)
         if dist is not None:
             dist.barrier()
-        ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return reduce_max(e0.elapsed_time(e1), dist, dev)
 
     with torch.cuda.stream(stream):
         sampler = ClockSampler(local)
         sampler.start()
         ms = timed(g, args.steps, args.warmup)
         clocks = sampler.stop()
+        ms_plain = timed(g_plain, args.steps, args.warmup)
     for x in layers:
         x.check()
+    del g_plain
 
     e2e = None
     if not args.no_e2e:
@@ -363,7 +395,7 @@ def gpu_arm(args):
         for x, oh in zip(layers, o_host):
             assert torch.equal(oh.view(torch.int16), x.out.cpu().view(torch.int16))
         qb = sum(q.numel() * 2 for q in q_host)
-        e2e = {"value": world * L * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+        e2e = {"value": aggregate_rate(world, L, args.steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": qb, "d2h_bytes_per_step": qb,
                "ms_per_step": ms_e2e / args.steps}
         del g2
@@ -383,7 +415,7 @@ def gpu_arm(args):
     traffic = recorded_traffic()
     line = {
         "metric": METRIC,
-        "value": world * L * args.steps / (ms / 1e3),
+        "value": aggregate_rate(world, L, args.steps, ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -401,7 +433,8 @@ def gpu_arm(args):
             "layers_per_step": L,
             "step": f"one decode token through {L} layers with distinct caches",
             "l2": f"inputs larger than L2: {L} distinct layer caches (~{L * 128 // 1024} GiB)",
-            "launch": "CUDA graph of fused score/select/attend launches, PDL",
+            "launch": "CUDA graph of fused score/select/attend launches, PDL, "
+                      "ABSP_STEP_EARLY_PREFETCH",
             "parallelism": f"dp{world} (independent layer stacks per GPU)",
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -412,6 +445,10 @@ def gpu_arm(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": L * args.steps,
+        "variants": {"plain": {"value": aggregate_rate(world, L, args.steps, ms_plain),
+                               "ms_per_step": ms_plain / args.steps,
+                               "note": "absp_decode_step, no reads before the previous "
+                                       "launch completes"}},
         "clocks": clocks,
         "rebuild": {"ms_per_layer": rebuild_ms, "bytes_per_layer": rb_bytes,
                     "achieved_gbs": rb_bytes / (rebuild_ms * 1e-3) / 1e9,
