@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
         "absp_decode_step_host": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
         "absp_check_device_error": (st, [c_void_p, c_size_t, c_void_p, P(c_int32)]),
+        "absp_build_quantize_noalloc": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p,
+                                             c_void_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -108,7 +110,7 @@ EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_row_offs
             "absp_select_capacity", "absp_workspace_init", "absp_build_centroids",
             "absp_quantize_centroids", "absp_score_select", "absp_sparse_decode",
             "absp_decode_step", "absp_decode_step_ex", "absp_decode_step_host",
-            "absp_check_device_error")
+            "absp_check_device_error", "absp_build_quantize_noalloc")
 
 
 def lib() -> ctypes.CDLL:
@@ -291,6 +293,14 @@ def absp_decode_step_host(kv: LayerKV, cent: Centroids, q_host: torch.Tensor, bu
     _check(_lib.absp_decode_step_host(kv.ref, cent.ref, _ptr(q_host), int(budget),
                                       _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)),
            "absp_decode_step_host")
+
+
+def absp_build_quantize_noalloc(kv: LayerKV, cent: Centroids, device_status=None,
+                                stream=None) -> None:
+    """Centroid build + INT4 quantisation without a caller workspace (the
+    library's static scratch array is used instead)."""
+    _check(_lib.absp_build_quantize_noalloc(kv.ref, cent.ref, _ptr(device_status),
+                                            _stream(stream)), "absp_build_quantize_noalloc")
 
 
 def absp_check_device_error(ws: torch.Tensor, stream=None):

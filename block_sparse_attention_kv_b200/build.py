@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libabsp.so")
-SOURCES = ["abi.cu", "centroids.cu", "decode.cu"]
+SOURCES = ["abi.cu", "centroids.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["absp_internal.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -20,8 +20,10 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+}  // namespace
+
 // Validate a layer description and fill the by-value kernel descriptor.
-absp_status make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v) {
+absp_status absp::make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v) {
     if (kv == nullptr || d == nullptr) return ABSP_ERR_INVALID_ARG;
     if (kv->head_dim != ABSP_HEAD_DIM || kv->page_size != ABSP_PAGE_SIZE)
         return ABSP_ERR_UNSUPPORTED;
@@ -66,6 +68,8 @@ absp_status make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v) {
     d->rows_per_seq = rows;
     return ABSP_OK;
 }
+
+namespace {
 
 absp_status check_budget(const KvDesc& d, int32_t budget, int32_t* kmax, int32_t* nmax) {
     if (budget < ABSP_PAGE_SIZE || budget > ABSP_MAX_BUDGET) return ABSP_ERR_INVALID_ARG;
@@ -134,13 +138,17 @@ absp_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
     return ABSP_OK;
 }
 
-absp_status check_cent(const absp_centroids* c) {
+}  // namespace
+
+absp_status absp::check_cent(const absp_centroids* c) {
     if (c == nullptr || c->codes == nullptr || c->scale == nullptr || c->zp == nullptr)
         return ABSP_ERR_INVALID_ARG;
     if (!aligned(c->codes, kAlign) || !aligned(c->scale, 4) || !aligned(c->zp, 4))
         return ABSP_ERR_INVALID_ARG;
     return ABSP_OK;
 }
+
+namespace {
 
 absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* cent,
                        const void* q, int32_t budget, int32_t* sel, int32_t* sel_count,

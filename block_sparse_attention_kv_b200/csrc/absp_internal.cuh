@@ -271,6 +271,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// ----------------------------------------------------- host validation --
+
+// Checks a layer description and fills the kernel descriptor (abi.cu).
+absp_status make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v);
+// Checks the three centroid buffers (abi.cu).
+absp_status check_cent(const absp_centroids* c);
+
 // ------------------------------------------------------------ launchers --
 
 // Build step (centroids.cu)

@@ -1,0 +1,79 @@
+// Allocation-free centroid build + INT4 quantisation.
+//
+// Some callers cannot allocate device memory at the point where they build
+// a layer's centroids: code that runs inside a host framework which owns
+// every device allocation through its own pool (an inference server, a
+// plugin of another runtime), or code on a path where a cudaMalloc is not
+// allowed or would synchronise the device.  absp_build_centroids needs a
+// caller-provided workspace; this entry point instead uses a scratch array
+// compiled into the library, so the caller only passes the layer (inputs)
+// and the centroid buffers (outputs).
+//
+// The scratch is a file-scope __device__ array of ABSP_NOALLOC_BUILD_WS_BYTES
+// bytes.  It lives in this file's own module: every GPU on which the module
+// is loaded (at the first call of the entry point on that GPU) holds it until
+// the process exits.  All calls on one GPU share it and it keeps the last
+// call's contents, so each call clears the parts that must start at zero
+// (the error word and the per-channel min/max keys), and calls whose work
+// overlaps on the GPU (different streams, no ordering between them) race on
+// it: the caller must order them.
+#include <mutex>
+
+#include "absp_internal.cuh"
+
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_build_ws[ABSP_NOALLOC_BUILD_WS_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_ws_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_ws_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_build_ws);
+        if (e != cudaSuccess) return e;
+        g_ws_ptr[dev] = p;
+    }
+    *out = g_ws_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" absp_status absp_build_quantize_noalloc(const absp_layer_kv* kv,
+                                                   const absp_centroids* out,
+                                                   int32_t* device_status, void* stream) {
+    absp::KvDesc d;
+    absp_status st = absp::make_desc(kv, &d, false);
+    if (st != ABSP_OK) return st;
+    if ((st = absp::check_cent(out)) != ABSP_OK) return st;
+    if (device_status != nullptr && (reinterpret_cast<uintptr_t>(device_status) % 4) != 0)
+        return ABSP_ERR_INVALID_ARG;
+    if (absp::build_ws_bytes(d) > static_cast<size_t>(ABSP_NOALLOC_BUILD_WS_BYTES))
+        return ABSP_ERR_UNSUPPORTED;
+    void* ws = nullptr;
+    if (noalloc_scratch(&ws) != cudaSuccess) return ABSP_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the error word and detail start at zero; launch_build resets the
+    // min/max keys itself
+    if (cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return ABSP_ERR_CUDA;
+    const absp::BuildWs w = absp::build_ws_layout(ws, d);
+    if (absp::launch_build(d, w, s) != cudaSuccess) return ABSP_ERR_CUDA;
+    if (absp::launch_quantize(d, w, out->codes, out->scale, out->zp, s) != cudaSuccess)
+        return ABSP_ERR_CUDA;
+    if (device_status != nullptr &&
+        cudaMemcpyAsync(device_status, ws, 2 * sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+        return ABSP_ERR_CUDA;
+    return ABSP_OK;
+}

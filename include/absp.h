@@ -204,6 +204,33 @@ ABSP_API absp_status absp_decode_step_host(const absp_layer_kv* kv,
                                   int32_t budget_tokens, void* out_host, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* Allocation-free steps 1-2.  The paper has no counterpart to this call;
+ * it exists for callers that cannot allocate device memory where they build
+ * a layer's centroids (code inside a framework that owns all device memory
+ * through its own pool, or on a path where cudaMalloc is forbidden or would
+ * synchronise the device).  Same results as absp_build_centroids followed
+ * by absp_quantize_centroids, but the workspace is a static array of
+ * ABSP_NOALLOC_BUILD_WS_BYTES bytes inside the library instead of a caller
+ * buffer; the caller passes only the layer and the centroid buffers.
+ *   - Layers whose absp_build_workspace_size exceeds that size are
+ *     rejected with ABSP_ERR_UNSUPPORTED before anything is launched.
+ *   - No device memory is allocated by the call.  The array itself is held
+ *     on every GPU where the library's static-scratch module is loaded (at
+ *     the first call on that GPU) until the process exits.
+ *   - The first call on each device looks the array's device address up on
+ *     the host (with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a GPU share the array; each call clears what must start
+ *     at zero.  Calls whose GPU work can overlap (unordered streams) race on
+ *     the array and must be ordered by the caller.
+ *   - device_status (optional, device memory, 2 x int32, may be NULL)
+ *     receives {error code, detail} of the device-side checks when the work
+ *     completes: 0 or ABSP_ERR_DEVICE_FAULT / ABSP_ERR_TIMEOUT. */
+#define ABSP_NOALLOC_BUILD_WS_BYTES (16u << 20)
+ABSP_API absp_status absp_build_quantize_noalloc(const absp_layer_kv* kv,
+                                                 const absp_centroids* out,
+                                                 int32_t* device_status, void* stream);
+
 /* Synchronises `stream`, reads the workspace's error word and clears it.
  * Returns ABSP_OK, ABSP_ERR_DEVICE_FAULT or ABSP_ERR_TIMEOUT; *detail (if
  * not NULL) receives the first faulting sequence/unit index. */

@@ -1,0 +1,73 @@
+"""The allocation-free centroid build against the workspace build.
+
+absp_build_quantize_noalloc serves callers that cannot allocate device
+memory when they build centroids (a host framework that owns all device
+memory, or a path where cudaMalloc is not allowed); it uses a static scratch
+array inside the library instead of a caller workspace.  Its INT4 codes,
+scales and zero points must equal those of absp_build_centroids +
+absp_quantize_centroids bit for bit, also on the second of two calls in a
+row (the shared scratch keeps the previous call's contents).
+
+This file sorts last so that a run stopping at the first failure has
+already run every other test.
+"""
+
+import pytest
+import torch
+
+from block_sparse_attention_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_kv_b200 import build
+    build.build()
+    from block_sparse_attention_kv_b200 import abi, pipeline
+    return abi, pipeline
+
+
+def test_noalloc_build_matches_workspace_build_on_two_calls(lib):
+    abi, pipeline = lib
+    # the first layer is the larger, so the second call runs over scratch
+    # left dirty by the first
+    cases = [synth.WORKLOADS["llama31_8b_32k"],
+             synth.custom("noalloc_ragged", 3, 12, 3, [4097, 900, 33], [16, 32, 64], 512,
+                          seed=77)]
+    for i, w in enumerate(cases):
+        d = synth.make_layer(w, i, "cuda")
+        ref = pipeline.DeviceLayer(d)
+        ref.build_centroids()                       # workspace entry points
+        cent = abi.alloc_centroids(ref.kv, d.q.device)
+        status = torch.full((2,), -1, dtype=torch.int32, device=d.q.device)
+        abi.absp_build_quantize_noalloc(ref.kv, cent, status)
+        torch.cuda.synchronize()
+        assert status.tolist() == [0, 0]
+        assert torch.equal(cent.codes, ref.cent.codes), w.name
+        assert torch.equal(cent.scale.view(torch.int32), ref.cent.scale.view(torch.int32))
+        assert torch.equal(cent.zp, ref.cent.zp)
+        # the decode path reads the allocation-free centroids like the others
+        out = torch.empty_like(d.q)
+        abi.absp_decode_step(ref.kv, cent, d.q, ref.budget, out, ref.ws)
+        ref.decode_step()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref.out.view(torch.int16))
+
+
+def test_noalloc_rejects_layers_beyond_its_scratch(lib):
+    abi, _ = lib
+    # 8 sequences x 128K tokens x 8 heads of 16-token blocks need far more
+    # than the static scratch: rejected on the host, nothing launched
+    w = synth.WORKLOADS["rebuild_8x128k"]
+    d = synth.make_layer(synth.custom("tiny_for_ptrs", 1, 8, 8, [16], [16] * 8, 64, seed=1),
+                         0, "cuda")
+    kv = abi.LayerKV(d.seq_lens, d.page_table, d.k_pages, d.v_pages, [16] * 8, 32)
+    kv.c.num_seqs = w.num_seqs
+    kv.c.max_pages_per_seq = w.ctx // 16
+    assert abi.absp_build_workspace_size(kv) > 16 << 20
+    cent = abi.alloc_centroids(abi.LayerKV(d.seq_lens, d.page_table, d.k_pages, d.v_pages,
+                                           [16] * 8, 32), d.q.device)
+    with pytest.raises(abi.AbspError) as e:
+        abi.absp_build_quantize_noalloc(kv, cent)
+    assert e.value.status == abi.ABSP_ERR_UNSUPPORTED
