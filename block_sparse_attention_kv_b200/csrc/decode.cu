@@ -138,7 +138,7 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v) {
 // order-preserving keys (keys > T are in, plus `rem` keys equal to T).
 __device__ __forceinline__ void radix_threshold(const float* sc, int n, int k, uint32_t* hist, Small& sm,
                                 uint32_t* T_out, int* rem_out) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     uint32_t prefix = 0, mask = 0;
     int rem = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
@@ -341,8 +341,12 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
     compact_by_threshold(sc, n, T, rem, out, sm);
 }
 
+#ifndef ABSP_DECODE_MIN_BLOCKS
+#define ABSP_DECODE_MIN_BLOCKS 2
+#endif
+
 template <int MODE, bool BIG_GROUP, bool EARLY>
-__global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
+__global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t smem_raw[];
@@ -422,7 +426,10 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         zpv = p.zp[pi];
     }
     if constexpr (EARLY) {
-        // only the query may be produced by the preceding kernel
+        // B0 only needs the cluster's CTAs to have started: wait for it while
+        // the preceding kernel still runs.  Only the query may be produced
+        // by the preceding kernel.
+        cluster_wait();
         pdl_wait();
         pdl_trigger();
     }
@@ -450,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
         const uint32_t scores_u32 = smem_u32(scores);
         const uint32_t bar_score = smem_u32(&sm.bar_score);
         float lmin = INFINITY, lmax = -INFINITY;
-        cluster_wait();  // B0: every CTA of the cluster is running
+        if constexpr (!EARLY) cluster_wait();  // B0: every CTA of the cluster is running
         {   // histogram bins of the select, zeroed while the codes stream in
             uint32_t* hist = reinterpret_cast<uint32_t*>(regB + p.scratch_off);
             for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
@@ -830,19 +837,24 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : 2)
                 return;
             }
             mbar_wait_bounded<true>(smem_u32(&sm.bar_merge), 0, p.err, 3);
+            // per (row, partial) weight exp2(m_r - M) / L, computed once
+            float* fac = Ow;                   // [G][C]; the warp partials are consumed
+            if (tid < G) {
+                float M = -INFINITY;
+                for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, partM[r * G + tid]);
+                float L = 0.0f;
+                if (M != -INFINITY)
+                    for (uint32_t r = 0; r < C; ++r) L += partL[r * G + tid] * exp2f(partM[r * G + tid] - M);
+                const float invL = L > 0.0f ? 1.0f / L : 0.0f;
+                for (uint32_t r = 0; r < C; ++r)
+                    fac[tid * C + r] = M != -INFINITY ? exp2f(partM[r * G + tid] - M) * invL : 0.0f;
+            }
+            __syncthreads();
             for (int idx = tid; idx < G * kD; idx += kThreads) {
                 const int row = idx >> 7, d = idx & (kD - 1);
-                float M = -INFINITY;
-                for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, partM[r * G + row]);
-                float L = 0.0f, Oacc = 0.0f;
-                if (M != -INFINITY) {
-                    for (uint32_t r = 0; r < C; ++r) {
-                        const float f = exp2f(partM[r * G + row] - M);
-                        L += partL[r * G + row] * f;
-                        Oacc += partO[(r * G + row) * kD + d] * f;
-                    }
-                }
-                outp[row * kD + d] = __float2bfloat16_rn(L > 0.0f ? Oacc / L : 0.0f);
+                float Oacc = 0.0f;
+                for (uint32_t r = 0; r < C; ++r) Oacc += partO[(r * G + row) * kD + d] * fac[row * C + r];
+                outp[row * kD + d] = __float2bfloat16_rn(Oacc);
             }
         }
     }
