@@ -52,7 +52,7 @@ constexpr int kMaxSlots = 2;                         // page buffers per warp
 constexpr int kBins = 1024;                          // value histogram
 constexpr int kMaxCand = 1024;                       // boundary-bin candidates
 constexpr int kMaxBitmapWords = (ABSP_MAX_BLOCKS_PER_HEAD + 31) / 32;
-constexpr int kSelectScratch = (kBins + 2 * kMaxCand + 2 * kMaxBitmapWords) * 4;
+constexpr int kSelectScratch = (kBins + 2 * kMaxCand + kMaxBitmapWords) * 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Params {
@@ -173,8 +173,8 @@ __device__ __forceinline__ void radix_threshold(const float* sc, int n, int k, u
 // Ordered compaction of the top-k by a threshold: keys > T are in, and of
 // the keys == T the `rem` lowest indices.  Each warp compacts a contiguous
 // index range 32 scores at a time with ballots.
-__device__ __forceinline__ void compact_by_threshold(const float* sc, int n, uint32_t T, int rem, int32_t* out,
-                                     Small& sm) {
+__device__ __forceinline__ void compact_by_threshold(const float* sc, int n, uint32_t T, int rem,
+                                                     int32_t* out, int lo, int hi, Small& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per_w = (n + kWarps - 1) / kWarps;
     const int w0 = min(n, warp * per_w), w1 = min(n, w0 + per_w);
@@ -199,52 +199,64 @@ __device__ __forceinline__ void compact_by_threshold(const float* sc, int n, uin
         const uint32_t bg = __ballot_sync(0xffffffffu, isg);
         const uint32_t be = __ballot_sync(0xffffffffu, ise);
         const uint32_t gp = gtb + __popc(bg & lt), ep = eqb + __popc(be & lt);
-        if (isg) out[gp + min(ep, r)] = i;
-        else if (ise && ep < r) out[gp + ep] = i;
+        int pos = -1;
+        if (isg) pos = static_cast<int>(gp + min(ep, r));
+        else if (ise && ep < r) pos = static_cast<int>(gp + ep);
+        if (pos >= lo && pos < hi) out[pos - lo] = i;
         gtb += __popc(bg);
         eqb += __popc(be);
     }
     __syncthreads();
 }
 
-// Ascending list of the set bits of bitmap[0..nwords), by one warp.
-__device__ __forceinline__ void warp_compact_bitmap(const uint32_t* bitmap, int nwords,
-                                                    int32_t* out) {
+// Entries [lo, hi) of the ascending list of the set bits of
+// bitmap[0..nwords), by one warp: out[pos - lo] = bit index.
+__device__ __forceinline__ void warp_extract_bitmap(const uint32_t* bitmap, int nwords,
+                                                    int32_t* out, int lo, int hi) {
     const int lane = threadIdx.x & 31;
     const int wpl = (nwords + 31) / 32;
     const int j0 = min(nwords, lane * wpl), j1 = min(nwords, j0 + wpl);
+    uint32_t words[16];
     uint32_t cnt = 0;
-    for (int j = j0; j < j1; ++j) cnt += __popc(bitmap[j]);
-    uint32_t pos = warp_excl_scan(cnt);
-    for (int j = j0; j < j1; ++j) {
-        uint32_t bits = bitmap[j];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        words[u] = j0 + u < j1 ? bitmap[j0 + u] : 0u;
+        cnt += __popc(words[u]);
+    }
+    int pos = static_cast<int>(warp_excl_scan(cnt));
+    if (pos + static_cast<int>(cnt) <= lo || pos >= hi) return;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        uint32_t bits = words[u];
         while (bits) {
             const int b = __ffs(bits) - 1;
-            out[pos++] = j * 32 + b;
+            if (pos >= lo && pos < hi) out[pos - lo] = (j0 + u) * 32 + b;
+            ++pos;
             bits &= bits - 1u;
         }
     }
 }
 
-// Top-k of sc[0..n) (largest scores, ties to the lower index), written to
-// out[0..k) in ascending index order; [mn, mx] is the range of the scores.
-// The kBins histogram bins at the start of `scratch` must be zero on entry.
-// n <= 65535.
-__device__ __forceinline__ void block_topk(const float* sc, int n, int k, float mn, float mx, int32_t* out,
-                           uint32_t* scratch, Small& sm) {
+// Top-k of sc[0..n) (largest scores, ties to the lower index) in ascending
+// index order; only list entries [lo, hi) are written, to out[0 .. hi-lo).
+// [mn, mx] is the range of the scores.  The kBins histogram bins at the
+// start of `scratch` must be zero on entry.  n <= 65535.
+__device__ __forceinline__ void block_topk(const float* sc, int n, int k, float mn, float mx,
+                                           int32_t* out, int lo, int hi, uint32_t* scratch,
+                                           Small& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (k >= n) {
-        for (int i = tid; i < n; i += kThreads) out[i] = i;
+        for (int i = max(0, lo) + tid; i < min(n, hi); i += kThreads) out[i - lo] = i;
         __syncthreads();
         return;
     }
     uint32_t* hist = scratch;
     uint32_t* ckey = scratch + kBins;
     int32_t* cidx = reinterpret_cast<int32_t*>(scratch + kBins + kMaxCand);
-    uint32_t* bitmap = scratch + kBins + 2 * kMaxCand;
+    uint32_t* inw = scratch + kBins + 2 * kMaxCand;
     const float inv = static_cast<float>(kBins) / (mx - mn);
     if (!(mx > mn)) {                 // every score equal: lowest k indices
-        compact_by_threshold(sc, n, order_key(mx), k, out, sm);
+        compact_by_threshold(sc, n, order_key(mx), k, out, lo, hi, sm);
         return;
     }
     if (inv < INFINITY) {
@@ -279,14 +291,15 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                     cum += c[j];
                 }
             }
+            if (tid == 32) sm.misc[3] = 0;
         }
         __syncthreads();
         const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
         if (m <= kMaxCand) {
-            // one pass: per 32 scores, a ballot word of the scores above bin
-            // bstar (in) and one of the scores inside it (candidates)
-            uint32_t* inw = bitmap;
-            uint32_t* eqw = bitmap + kMaxBitmapWords;
+            // one pass: a ballot word per 32 scores marks those above bin
+            // bstar (selected); the scores inside bstar become candidates,
+            // all of them selected when the whole bin is needed
+            const bool all_in = need == m;
             const int nwords = (n + 31) / 32;
             constexpr int V = 8;
             for (int w0 = warp; w0 < nwords; w0 += kWarps * V) {
@@ -299,37 +312,36 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     const int wd = w0 + v * kWarps;
-                    const bool live = wd < nwords && wd * 32 + lane < n;
+                    const int i = wd * 32 + lane;
+                    const bool live = wd < nwords && i < n;
                     const int bn = value_bin(x[v], mn, inv);
-                    const uint32_t gw = __ballot_sync(0xffffffffu, live && bn > bstar);
-                    const uint32_t ew = __ballot_sync(0xffffffffu, live && bn == bstar);
-                    if (lane == 0 && wd < nwords) {
-                        inw[wd] = gw;
-                        eqw[wd] = ew;
+                    const uint32_t gw =
+                        __ballot_sync(0xffffffffu, live && (bn > bstar || (all_in && bn == bstar)));
+                    if (lane == 0 && wd < nwords) inw[wd] = gw;
+                    if (!all_in && live && bn == bstar) {
+                        const int pos = atomicAdd(&sm.misc[3], 1);
+                        ckey[pos] = order_key(x[v]);
+                        cidx[pos] = i;
                     }
                 }
             }
             __syncthreads();
-            if (warp == 0) {
-                // warp 0: list the candidates, rank them exactly (ties to the
-                // lower index), add the `need` best to the bitmap, compact
-                warp_compact_bitmap(eqw, nwords, cidx);
-                __syncwarp();
-                for (int c = lane; c < m; c += 32) ckey[c] = order_key(sc[cidx[c]]);
-                __syncwarp();
-                for (int c = lane; c < m; c += 32) {
+            if (!all_in) {
+                // exact rank among the candidates: larger key first, ties to
+                // the lower index; the `need` best join the selection
+                for (int c = tid; c < m; c += kThreads) {
                     const uint32_t key = ckey[c];
                     const int idx = cidx[c];
                     int rank = 0;
                     for (int j = 0; j < m; ++j) {
                         const uint32_t kj = ckey[j];
-                        rank += (kj > key) || (kj == key && j < c);   // cidx ascending
+                        rank += (kj > key) || (kj == key && cidx[j] < idx);
                     }
                     if (rank < need) atomicOr(&inw[idx >> 5], 1u << (idx & 31));
                 }
-                __syncwarp();
-                warp_compact_bitmap(inw, nwords, out);
+                __syncthreads();
             }
+            if (warp == 0) warp_extract_bitmap(inw, nwords, out, lo, hi);
             __syncthreads();
             return;
         }
@@ -338,7 +350,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
     uint32_t T = 0;
     int rem = 0;
     radix_threshold(sc, n, k, scratch, sm, &T, &rem);
-    compact_by_threshold(sc, n, T, rem, out, sm);
+    compact_by_threshold(sc, n, T, rem, out, lo, hi, sm);
 }
 
 #ifndef ABSP_DECODE_MIN_BLOCKS
@@ -434,6 +446,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         pdl_trigger();
     }
     int K = 0;
+    int sel_lo = 0, sel_hi = 0;  // list entries held in sel_s
 
     if constexpr (kSelect) {
         // ---------------------------------------------------- A: score --
@@ -554,11 +567,23 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             smin = fminf(smin, sm.cmm[r].x);
             smax = fmaxf(smax, sm.cmm[r].y);
         }
-        block_topk(scores, n, K, smin, smax, sel_s,
+        if (MODE == kModeSelect) {
+            sel_lo = 0;
+            sel_hi = K;
+        } else {
+            // this CTA attends list entries [sel_lo, sel_hi): the blocks of
+            // its share [pb, pe) of the K * bs/16 selected pages
+            const int P = K * spb;
+            const int pb = static_cast<int>((static_cast<int64_t>(P) * rank) / C);
+            const int pe = static_cast<int>((static_cast<int64_t>(P) * (rank + 1)) / C);
+            sel_lo = pb / spb;
+            sel_hi = pe > pb ? (pe - 1) / spb + 1 : sel_lo;
+        }
+        block_topk(scores, n, K, smin, smax, sel_s, sel_lo, sel_hi,
                    reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm);
         if (MODE == kModeSelect) {
             int32_t* dst = p.sel + (static_cast<int64_t>(s) * Hkv + h) * p.kmax;
-            for (int i = tid; i < K; i += kThreads) dst[i] = sel_s[i];
+            for (int i = tid; i < K; i += kThreads) dst[i] = sel_s[i];  // [0, K) held
             if (tid == 0) p.sel_count[static_cast<int64_t>(s) * Hkv + h] = K;
             return;
         }
@@ -615,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             int valid = 0;
             if (lane == 0) {
                 const int j = pb + warp + kWarps * i;
-                const int b = sel_s[j / spb];
+                const int b = sel_s[j / spb - sel_lo];
                 int phys = -1;
                 if (b >= 0) {
                     const int lp = b * spb + (j % spb);
