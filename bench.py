@@ -66,6 +66,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
     return ap.parse_args()
 
 
@@ -147,15 +148,16 @@ def recorded_traffic():
     return None
 
 
-def step_bytes(d, sel, cnt):
+def step_bytes(d, sel, cnt, block_size=None):
     """Algorithmic bytes of one decode layer-step of layer data `d`."""
     lens = d.seq_lens.cpu().numpy()
     S, Hkv, Hq = d.num_seqs, d.num_kv_heads, d.num_q_heads
+    bsz = d.block_size if block_size is None else block_size
     total = S * Hq * 128 * 2 * 2                       # q in + out
     for s in range(S):
         L = int(lens[s])
         for h in range(Hkv):
-            bs = int(d.block_size[h])
+            bs = int(bsz[h])
             n = (L + bs - 1) // bs
             total += n * 64 + 128 * 8                  # codes + scale/zp
             toks = 0
@@ -196,6 +198,37 @@ def reduce_max(value: float, dist=None, device=None) -> float:
 def aggregate_rate(world: int, layers: int, steps: int, ms: float) -> float:
     """Whole-job layer-steps/s: all ranks' layer-steps over the max time."""
     return world * layers * steps / (ms / 1e3)
+
+
+def rebuild_large(dev, stream, abi, pipeline, synth):
+    """Steps 1-2 at batch 8 x 131072 tokens (8 KV heads, mixed block sizes)."""
+    w = synth.WORKLOADS["rebuild_8x128k"]
+    with torch.cuda.stream(stream):
+        d = synth.make_layer(w, 0, dev)
+        y = pipeline.DeviceLayer(d, stream=stream.cuda_stream)
+    ws = abi.alloc_workspace(abi.absp_build_workspace_size(y.kv), dev)
+    sc = stream.cuda_stream
+    for _ in range(2):
+        abi.absp_build_centroids(y.kv, ws, sc)
+        abi.absp_quantize_centroids(y.kv, ws, y.cent, sc)
+    stream.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = 5
+    e0.record(stream)
+    for _ in range(reps):
+        abi.absp_build_centroids(y.kv, ws, sc)
+        abi.absp_quantize_centroids(y.kv, ws, y.cent, sc)
+    e1.record(stream)
+    stream.synchronize()
+    st, _ = abi.absp_check_device_error(ws, sc)
+    assert st == abi.ABSP_OK
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = rebuild_bytes(d)
+    del y, d, ws
+    torch.cuda.empty_cache()
+    return {"workload": "rebuild_8x128k: 8 sequences x 131072 tokens, 8 KV heads",
+            "ms": ms, "bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9}
 
 
 # ------------------------------------------------------- CPU oracle leg --
@@ -322,6 +355,7 @@ def gpu_arm(args):
     assert st == abi.ABSP_OK, "device fault while building centroids"
     rb_bytes = sum(rebuild_bytes(x.data) for x in layers) / L
     del bws
+    rb_large = None if args.no_variants else rebuild_large(dev, stream, abi, pipeline, synth)
 
     # algorithmic bytes from each layer's own selection
     nbytes = []
@@ -378,6 +412,46 @@ def gpu_arm(args):
     for x in layers:
         x.check()
     del g_plain
+
+    # fixed block size for every KV head (the uniform-block methods the page
+    # compares against), same caches, queries and token budget
+    fixed = {}
+    if not args.no_variants:
+        big = abi.LayerKV(  # the largest centroid table: block size 16 everywhere
+                          layers[0].data.seq_lens, layers[0].data.page_table,
+                          layers[0].data.k_pages, layers[0].data.v_pages,
+                          [16] * layers[0].data.num_kv_heads, layers[0].data.num_q_heads)
+        fws = abi.alloc_workspace(abi.absp_build_workspace_size(big), dev)
+        for bsz in (16, 32, 64):
+            vl = [pipeline.DeviceLayer(x.data, block_size=[bsz] * x.data.num_kv_heads,
+                                       stream=sc) for x in layers]
+            vb = []
+            for y in vl:
+                abi.absp_build_centroids(y.kv, fws, sc)
+                abi.absp_quantize_centroids(y.kv, fws, y.cent, sc)
+                y.score_select()
+                stream.synchronize()
+                vb.append(step_bytes(y.data, y.sel.cpu().numpy(), y.sel_count.cpu().numpy(),
+                                     y.block_size))
+                abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws, EARLY, sc)
+            stream.synchronize()
+            gv = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gv, stream=stream):
+                for y in vl:
+                    abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws,
+                                            EARLY, sc)
+            with torch.cuda.stream(stream):
+                ms_v = timed(gv, args.steps, args.warmup)
+            for y in vl:
+                y.check()
+            bpl = float(np.mean(vb))
+            fixed[f"fixed_block_{bsz}"] = {
+                "value": aggregate_rate(world, L, args.steps, ms_v),
+                "ms_per_step": ms_v / args.steps,
+                "bytes_per_launch": bpl,
+                "achieved_gbs": bpl / (ms_v / (args.steps * L) * 1e-3) / 1e9}
+            del gv, vl
+        del fws
 
     e2e = None
     if not args.no_e2e:
@@ -445,14 +519,16 @@ def gpu_arm(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": L * args.steps,
-        "variants": {"plain": {"value": aggregate_rate(world, L, args.steps, ms_plain),
+        "variants": {**fixed, "plain": {"value": aggregate_rate(world, L, args.steps, ms_plain),
                                "ms_per_step": ms_plain / args.steps,
                                "note": "absp_decode_step, no reads before the previous "
                                        "launch completes"}},
         "clocks": clocks,
         "rebuild": {"ms_per_layer": rebuild_ms, "bytes_per_layer": rb_bytes,
                     "achieved_gbs": rb_bytes / (rebuild_ms * 1e-3) / 1e9,
-                    "frac": rb_bytes / (rebuild_ms * 1e-3) / 1e9 / peak},
+                    "frac": rb_bytes / (rebuild_ms * 1e-3) / 1e9 / peak,
+                    "large": None if rb_large is None else
+                    {**rb_large, "frac": rb_large["achieved_gbs"] / peak}},
     }
     del g
     if rank == 0:

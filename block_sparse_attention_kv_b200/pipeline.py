@@ -13,12 +13,16 @@ from . import abi
 
 
 class DeviceLayer:
-    def __init__(self, data, budget: int = None, stream=None):
-        """`data` is a synth.LayerData on a CUDA device."""
+    def __init__(self, data, budget: int = None, stream=None, block_size=None):
+        """`data` is a synth.LayerData on a CUDA device; `block_size`
+        overrides its per-KV-head block-size table (same cache, other
+        blocking)."""
         self.data = data
         self.device = data.q.device
         self.budget = int(budget if budget is not None else data.budget)
-        self.kv = abi.LayerKV.from_layer(data)
+        self.block_size = list(data.block_size if block_size is None else block_size)
+        self.kv = abi.LayerKV(data.seq_lens, data.page_table, data.k_pages, data.v_pages,
+                              self.block_size, data.num_q_heads)
         self.cent = abi.alloc_centroids(self.kv, self.device)
         self.build_ws = None
         dws = abi.absp_decode_workspace_size(self.kv, self.budget)
