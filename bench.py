@@ -148,7 +148,7 @@ def recorded_traffic():
     return None
 
 
-def step_bytes(d, sel, cnt, block_size=None):
+def step_bytes(d, sel, cnt, block_size=None, bf16=False):
     """Algorithmic bytes of one decode layer-step of layer data `d`."""
     lens = d.seq_lens.cpu().numpy()
     S, Hkv, Hq = d.num_seqs, d.num_kv_heads, d.num_q_heads
@@ -159,7 +159,7 @@ def step_bytes(d, sel, cnt, block_size=None):
         for h in range(Hkv):
             bs = int(bsz[h])
             n = (L + bs - 1) // bs
-            total += n * 64 + 128 * 8                  # codes + scale/zp
+            total += n * 256 if bf16 else n * 64 + 128 * 8   # centroid rows (+ scale/zp)
             toks = 0
             for b in sel[s, h, :cnt[s, h]]:
                 toks += min(bs, L - int(b) * bs)
@@ -414,7 +414,8 @@ def gpu_arm(args):
     del g_plain
 
     # fixed block size for every KV head (the uniform-block methods the page
-    # compares against), same caches, queries and token budget
+    # compares against) and unquantised bf16 centroids (its precision
+    # baseline), on the same caches, queries and token budget
     fixed = {}
     if not args.no_variants:
         big = abi.LayerKV(  # the largest centroid table: block size 16 everywhere
@@ -422,9 +423,13 @@ def gpu_arm(args):
                           layers[0].data.k_pages, layers[0].data.v_pages,
                           [16] * layers[0].data.num_kv_heads, layers[0].data.num_q_heads)
         fws = abi.alloc_workspace(abi.absp_build_workspace_size(big), dev)
-        for bsz in (16, 32, 64):
-            vl = [pipeline.DeviceLayer(x.data, block_size=[bsz] * x.data.num_kv_heads,
-                                       stream=sc) for x in layers]
+        cases = [(f"fixed_block_{b}", b, abi.ABSP_CENTROIDS_INT4) for b in (16, 32, 64)]
+        cases.append(("bf16_centroids", None, abi.ABSP_CENTROIDS_BF16))
+        for name, bsz, fmt in cases:
+            vl = [pipeline.DeviceLayer(
+                x.data, stream=sc, fmt=fmt,
+                block_size=None if bsz is None else [bsz] * x.data.num_kv_heads)
+                for x in layers]
             vb = []
             for y in vl:
                 abi.absp_build_centroids(y.kv, fws, sc)
@@ -432,7 +437,7 @@ def gpu_arm(args):
                 y.score_select()
                 stream.synchronize()
                 vb.append(step_bytes(y.data, y.sel.cpu().numpy(), y.sel_count.cpu().numpy(),
-                                     y.block_size))
+                                     y.block_size, fmt == abi.ABSP_CENTROIDS_BF16))
                 abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws, EARLY, sc)
             stream.synchronize()
             gv = torch.cuda.CUDAGraph()
@@ -445,7 +450,7 @@ def gpu_arm(args):
             for y in vl:
                 y.check()
             bpl = float(np.mean(vb))
-            fixed[f"fixed_block_{bsz}"] = {
+            fixed[name] = {
                 "value": aggregate_rate(world, L, args.steps, ms_v),
                 "ms_per_step": ms_v / args.steps,
                 "bytes_per_launch": bpl,

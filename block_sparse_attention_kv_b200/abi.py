@@ -27,6 +27,8 @@ ABSP_ERR_DEVICE_FAULT = 4
 ABSP_ERR_TIMEOUT = 5
 
 ABSP_STEP_EARLY_PREFETCH = 1
+ABSP_CENTROIDS_INT4 = 0
+ABSP_CENTROIDS_BF16 = 1
 
 HEAD_DIM = 128
 PAGE_SIZE = 16
@@ -61,6 +63,7 @@ class absp_centroids(Structure):
         ("codes", POINTER(c_uint8)),
         ("scale", c_void_p),
         ("zp", c_void_p),
+        ("format", c_int32),
     ]
 
 
@@ -75,6 +78,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "absp_status_string": (c_char_p, [st]),
         "absp_centroid_sizes": (st, [P(absp_layer_kv), P(c_size_t), P(c_size_t), P(c_size_t)]),
+        "absp_centroid_sizes_fmt": (st, [P(absp_layer_kv), c_int32, P(c_size_t), P(c_size_t),
+                                         P(c_size_t)]),
         "absp_centroid_row_offset": (st, [P(absp_layer_kv), c_int32, c_int32, P(c_int64)]),
         "absp_build_workspace_size": (st, [P(absp_layer_kv), P(c_size_t)]),
         "absp_decode_workspace_size": (st, [P(absp_layer_kv), c_int32, P(c_size_t)]),
@@ -105,7 +110,8 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_row_offset",
+EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_sizes_fmt",
+            "absp_centroid_row_offset",
             "absp_build_workspace_size", "absp_decode_workspace_size",
             "absp_select_capacity", "absp_workspace_init", "absp_build_centroids",
             "absp_quantize_centroids", "absp_score_select", "absp_sparse_decode",
@@ -174,27 +180,29 @@ class LayerKV:
 
 
 class Centroids:
-    """Owns an absp_centroids over three device tensors."""
+    """Owns an absp_centroids over its device tensors."""
 
-    def __init__(self, codes: torch.Tensor, scale: torch.Tensor, zp: torch.Tensor):
-        self.codes, self.scale, self.zp = codes, scale, zp
+    def __init__(self, codes: torch.Tensor, scale: torch.Tensor, zp: torch.Tensor,
+                 fmt: int = ABSP_CENTROIDS_INT4):
+        self.codes, self.scale, self.zp, self.format = codes, scale, zp, int(fmt)
         self.c = absp_centroids(codes=ctypes.cast(codes.data_ptr(), POINTER(c_uint8)),
-                                scale=scale.data_ptr(), zp=zp.data_ptr())
+                                scale=scale.data_ptr() if scale.numel() else None,
+                                zp=zp.data_ptr() if zp.numel() else None, format=int(fmt))
 
     @property
     def ref(self):
         return ctypes.byref(self.c)
 
 
-def alloc_centroids(kv: LayerKV, device) -> Centroids:
-    """Device buffers sized by absp_centroid_sizes (torch owns the memory)."""
-    cb, sb, zb = absp_centroid_sizes(kv)
+def alloc_centroids(kv: LayerKV, device, fmt: int = ABSP_CENTROIDS_INT4) -> Centroids:
+    """Device buffers sized by absp_centroid_sizes_fmt (torch owns the memory)."""
+    cb, sb, zb = absp_centroid_sizes_fmt(kv, fmt)
     codes = torch.zeros(max(cb, 256) + 256, dtype=torch.uint8, device=device)
     off = (-codes.data_ptr()) % 256
     codes = codes[off:off + cb]
     scale = torch.zeros(sb // 4, dtype=torch.float32, device=device)
     zp = torch.zeros(zb // 4, dtype=torch.int32, device=device)
-    return Centroids(codes, scale, zp)
+    return Centroids(codes, scale, zp, fmt)
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
@@ -214,6 +222,13 @@ def absp_centroid_sizes(kv: LayerKV):
     a, b, c = c_size_t(), c_size_t(), c_size_t()
     _check(_lib.absp_centroid_sizes(kv.ref, ctypes.byref(a), ctypes.byref(b),
                                     ctypes.byref(c)), "absp_centroid_sizes")
+    return a.value, b.value, c.value
+
+
+def absp_centroid_sizes_fmt(kv: LayerKV, fmt: int):
+    a, b, c = c_size_t(), c_size_t(), c_size_t()
+    _check(_lib.absp_centroid_sizes_fmt(kv.ref, int(fmt), ctypes.byref(a), ctypes.byref(b),
+                                        ctypes.byref(c)), "absp_centroid_sizes_fmt")
     return a.value, b.value, c.value
 
 

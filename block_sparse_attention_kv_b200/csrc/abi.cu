@@ -141,9 +141,12 @@ absp_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
 }  // namespace
 
 absp_status absp::check_cent(const absp_centroids* c) {
-    if (c == nullptr || c->codes == nullptr || c->scale == nullptr || c->zp == nullptr)
+    if (c == nullptr || c->codes == nullptr) return ABSP_ERR_INVALID_ARG;
+    if (c->format != ABSP_CENTROIDS_INT4 && c->format != ABSP_CENTROIDS_BF16)
         return ABSP_ERR_INVALID_ARG;
-    if (!aligned(c->codes, kAlign) || !aligned(c->scale, 4) || !aligned(c->zp, 4))
+    if (!aligned(c->codes, kAlign)) return ABSP_ERR_INVALID_ARG;
+    if (c->format == ABSP_CENTROIDS_INT4 &&
+        (c->scale == nullptr || c->zp == nullptr || !aligned(c->scale, 4) || !aligned(c->zp, 4)))
         return ABSP_ERR_INVALID_ARG;
     return ABSP_OK;
 }
@@ -180,6 +183,7 @@ absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* 
     a.codes = cent ? cent->codes : nullptr;
     a.scale = cent ? cent->scale : nullptr;
     a.zp = cent ? cent->zp : nullptr;
+    a.cfmt = cent ? cent->format : ABSP_CENTROIDS_INT4;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.out = static_cast<__nv_bfloat16*>(out);
     a.sel = sel;
@@ -216,6 +220,22 @@ absp_status absp_centroid_sizes(const absp_layer_kv* kv, size_t* codes_bytes,
     if (st != ABSP_OK) return st;
     const size_t params = static_cast<size_t>(d.S) * d.Hkv * ABSP_HEAD_DIM * 4;
     if (codes_bytes) *codes_bytes = static_cast<size_t>(d.S) * d.rows_per_seq * ABSP_CODE_ROW_BYTES;
+    if (scale_bytes) *scale_bytes = params;
+    if (zp_bytes) *zp_bytes = params;
+    return ABSP_OK;
+}
+
+absp_status absp_centroid_sizes_fmt(const absp_layer_kv* kv, int32_t format,
+                                    size_t* codes_bytes, size_t* scale_bytes, size_t* zp_bytes) {
+    if (format != ABSP_CENTROIDS_INT4 && format != ABSP_CENTROIDS_BF16) return ABSP_ERR_INVALID_ARG;
+    KvDesc d;
+    absp_status st = make_desc(kv, &d, false);
+    if (st != ABSP_OK) return st;
+    const bool bf = format == ABSP_CENTROIDS_BF16;
+    const size_t params = bf ? 0 : static_cast<size_t>(d.S) * d.Hkv * ABSP_HEAD_DIM * 4;
+    if (codes_bytes)
+        *codes_bytes = static_cast<size_t>(d.S) * d.rows_per_seq * (bf ? 2 * ABSP_HEAD_DIM
+                                                                      : ABSP_CODE_ROW_BYTES);
     if (scale_bytes) *scale_bytes = params;
     if (zp_bytes) *zp_bytes = params;
     return ABSP_OK;
@@ -282,7 +302,7 @@ absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws, size_t ws
     if ((st = check_ws(ws, ws_bytes, build_ws_bytes(d))) != ABSP_OK) return st;
     if ((st = check_cent(out)) != ABSP_OK) return st;
     return from_cuda(launch_quantize(d, build_ws_layout(ws, d), out->codes, out->scale, out->zp,
-                                     static_cast<cudaStream_t>(stream)));
+                                     out->format, static_cast<cudaStream_t>(stream)));
 }
 
 absp_status absp_score_select(const absp_layer_kv* kv, const absp_centroids* cent, const void* q,

@@ -289,8 +289,9 @@ struct BuildWs {
 BuildWs build_ws_layout(void* ws, const KvDesc& kv);
 size_t build_ws_bytes(const KvDesc& kv);
 cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st);
+// format: ABSP_CENTROIDS_INT4 (codes + scale + zp) or ABSP_CENTROIDS_BF16
 cudaError_t launch_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
-                            int32_t* zp, cudaStream_t st);
+                            int32_t* zp, int format, cudaStream_t st);
 
 // Decode steps (decode.cu)
 enum DecodeMode : int { kModeSelect = 1, kModeAttend = 2, kModeFull = 3 };
@@ -308,6 +309,7 @@ struct DecodeArgs {
     int32_t budget;
     int32_t* err;
     int32_t nmax;                 // bound on blocks per head for this layer
+    int32_t cfmt;                 // centroid format (ABSP_CENTROIDS_*)
 };
 // early_prefetch: codes, parameters, lengths and page table are read before
 // the programmatic-dependency wait (only the query after it).

@@ -15,7 +15,8 @@
 //   quantize: reads the fp64 centroids back, derives scale / zero point from
 //             the min / max (fp64, IEEE division, rint half-to-even) and
 //             writes packed nibbles: lane L writes 2 bytes of each 64-byte
-//             row.
+//             row.  The BF16 store (the unquantised precision of Fig. 13)
+//             instead writes each centroid rounded to bf16, 256-byte rows.
 #include "absp_internal.cuh"
 
 namespace absp {
@@ -214,6 +215,40 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
     }
 }
 
+// fp64 -> bf16, round to nearest even, without double rounding: first round
+// to odd into fp32 (truncate, then set the last bit when inexact; fp32 keeps
+// 16 more bits than bf16), then round to nearest even into bf16.
+__device__ __forceinline__ uint32_t f64_to_bf16_rne(double x) {
+    const float f = __double2float_rz(x);
+    uint32_t u = __float_as_uint(f);
+    if (static_cast<double>(f) != x) u |= 1u;
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return u >> 16;
+}
+
+// BF16 centroid store: every fp64 centroid rounded to bf16, 256-byte rows.
+__global__ void __launch_bounds__(kBuildWarps * 32)
+    centroid_bf16_kernel(const KvDesc kv, BuildWs w, uint8_t* __restrict__ rows_out) {
+    const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int len = checked_len(kv, s, w.err);
+    const int tok0 = chunk * kChunkTokens;
+    if (len <= tok0) return;  // uniform over the CTA
+    const int bs = kv.bs[h];
+    const int n = (len + bs - 1) / bs;
+    const int b_begin = tok0 / bs;
+    const int b_end = min(n, (tok0 + kChunkTokens) / bs);
+    const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h];
+    for (int b = b_begin + warp; b < b_end; b += kBuildWarps) {
+        const double2* src = reinterpret_cast<const double2*>(w.cent + (row0 + b) * kD + lane * 4);
+        const double2 u = src[0], v = src[1];
+        uint2 o;
+        o.x = f64_to_bf16_rne(u.x) | (f64_to_bf16_rne(u.y) << 16);
+        o.y = f64_to_bf16_rne(v.x) | (f64_to_bf16_rne(v.y) << 16);
+        *reinterpret_cast<uint2*>(rows_out + (row0 + b) * (2 * kD) + lane * 8) = o;
+    }
+}
+
 }  // namespace
 
 size_t build_ws_bytes(const KvDesc& kv) {
@@ -250,8 +285,12 @@ cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st) {
 }
 
 cudaError_t launch_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
-                            int32_t* zp, cudaStream_t st) {
-    centroid_quantize_kernel<<<chunk_grid(kv), kBuildWarps * 32, 0, st>>>(kv, w, codes, scale, zp);
+                            int32_t* zp, int format, cudaStream_t st) {
+    if (format == ABSP_CENTROIDS_BF16)
+        centroid_bf16_kernel<<<chunk_grid(kv), kBuildWarps * 32, 0, st>>>(kv, w, codes);
+    else
+        centroid_quantize_kernel<<<chunk_grid(kv), kBuildWarps * 32, 0, st>>>(kv, w, codes, scale,
+                                                                           zp);
     return cudaGetLastError();
 }
 

@@ -357,7 +357,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 #define ABSP_DECODE_MIN_BLOCKS 2
 #endif
 
-template <int MODE, bool BIG_GROUP, bool EARLY>
+template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C>
 __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
@@ -382,6 +382,9 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     const int32_t* pt = p.kv.page_table + static_cast<int64_t>(s) * p.kv.max_pages;
     constexpr bool kSelect = (MODE & kModeSelect) != 0;
     constexpr bool kAttend = (MODE & kModeAttend) != 0;
+    // centroid rows: 64 B of INT4 codes, or 256 B of bf16 centroids
+    constexpr int kRow = BF16C ? 2 * kD : kRowBytes;
+    constexpr int kSRows = kStageBytes / kRow;         // rows per bulk stage
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
@@ -406,19 +409,19 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     const int per = ((n + static_cast<int>(C) - 1) / static_cast<int>(C) + 3) & ~3;
     const int r0 = min(n, static_cast<int>(rank) * per);
     const int nrows = min(n, r0 + per) - r0;
-    const int nchunks = (nrows + kStageRows - 1) / kStageRows;
+    const int nchunks = (nrows + kSRows - 1) / kSRows;
     const uint8_t* cbase =
-        p.codes + (static_cast<int64_t>(s) * p.kv.rows_per_seq + p.kv.row_base[h] + r0) * kRowBytes;
+        p.codes + (static_cast<int64_t>(s) * p.kv.rows_per_seq + p.kv.row_base[h] + r0) * kRow;
     if (tid == 0) {
         if (kSelect && (MODE != kModeSelect || rank == 0))
             mbar_arrive_expect_tx(smem_u32(&sm.bar_score), 16 * ((n + 3) / 4) + 8 * C);
         if (kSelect) {
             for (int c = 0; c < min(nchunks, kStages); ++c) {
-                const int rows = min(kStageRows, nrows - c * kStageRows);
+                const int rows = min(kSRows, nrows - c * kSRows);
                 const uint32_t bar = smem_u32(&sm.bar_code[c]);
-                mbar_arrive_expect_tx(bar, rows * kRowBytes);
+                mbar_arrive_expect_tx(bar, rows * kRow);
                 bulk_g2s(smem_u32(regA + c * kStageBytes), cbase + c * kStageBytes,
-                         rows * kRowBytes, bar);
+                         rows * kRow, bar);
             }
         }
     }
@@ -434,8 +437,10 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     int32_t zpv = 0;
     if (kSelect && tid < kD) {
         const int64_t pi = (static_cast<int64_t>(s) * Hkv + h) * kD + tid;
-        scl = p.scale[pi];
-        zpv = p.zp[pi];
+        if constexpr (!BF16C) {
+            scl = p.scale[pi];
+            zpv = p.zp[pi];
+        }
     }
     if constexpr (EARLY) {
         // B0 only needs the cluster's CTAs to have started: wait for it while
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             const __nv_bfloat16* qh = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD + tid;
             float qb = 0.0f;
             for (int j = 0; j < G; ++j) qb += __bfloat162float(qh[j * kD]);
-            sm.w[tid] = qb * scl;
+            sm.w[tid] = BF16C ? qb : qb * scl;
             sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
         }
         __syncthreads();
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         for (int c = 0; c < nchunks; ++c) {
             const int stage = c % kStages;
             mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / kStages) & 1, p.err, 1);
-            const int rows = min(kStageRows, nrows - c * kStageRows);
+            const int rows = min(kSRows, nrows - c * kSRows);
             const uint8_t* sbuf = regA + stage * kStageBytes;
             // each 8-lane group scores 4 consecutive rows
             for (int rb = 0; rb < rows; rb += 4 * (kThreads / 8)) {
@@ -487,20 +492,36 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int r = r4 + u;
-                    uint2 x = make_uint2(0u, 0u);
-                    if (r < rows) x = *reinterpret_cast<const uint2*>(sbuf + r * kRowBytes + sub * 8);
                     float acc = 0.0f;
+                    if constexpr (BF16C) {
+                        // 16 bf16 centroid channels per lane: score += qbar * c
+                        uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
+                        if (r < rows) {
+                            const uint4* src = reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
+                            y0 = src[0];
+                            y1 = src[1];
+                        }
+                        const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float f =
-                            __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
-                        acc = fmaf(wr[k], f, acc);
-                    }
+                        for (int k = 0; k < 8; ++k) {
+                            acc = fmaf(wr[2 * k], bf16lo(yy[k]), acc);
+                            acc = fmaf(wr[2 * k + 1], bf16hi(yy[k]), acc);
+                        }
+                    } else {
+                        uint2 x = make_uint2(0u, 0u);
+                        if (r < rows) x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float f =
-                            __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
-                        acc = fmaf(wr[8 + k], f, acc);
+                        for (int k = 0; k < 8; ++k) {
+                            const float f =
+                                __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
+                            acc = fmaf(wr[k], f, acc);
+                        }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float f =
+                                __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
+                            acc = fmaf(wr[8 + k], f, acc);
+                        }
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -512,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                     }
                 }
                 if (r4 < rows) {
-                    const uint32_t off = 4u * static_cast<uint32_t>(r0 + c * kStageRows + r4);
+                    const uint32_t off = 4u * static_cast<uint32_t>(r0 + c * kSRows + r4);
                     if (MODE == kModeSelect) {
                         if (sub == 0)
                             st_async_v4(dsmem_addr(scores_u32 + off, 0), q4[0], q4[1], q4[2],
@@ -527,12 +548,12 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             __syncthreads();
             if (tid == 0 && c + kStages < nchunks) {
                 const int cn = c + kStages;
-                const int rows_n = min(kStageRows, nrows - cn * kStageRows);
+                const int rows_n = min(kSRows, nrows - cn * kSRows);
                 const uint32_t bar = smem_u32(&sm.bar_code[stage]);
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(bar, rows_n * kRowBytes);
+                mbar_arrive_expect_tx(bar, rows_n * kRow);
                 bulk_g2s(smem_u32(regA + stage * kStageBytes), cbase + cn * kStageBytes,
-                         rows_n * kRowBytes, bar);
+                         rows_n * kRow, bar);
             }
         }
         // this CTA's score range, sent along with the scores
@@ -885,11 +906,11 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     }
 }
 
-template <int MODE, bool BIG, bool EARLY>
+template <int MODE, bool BIG, bool EARLY, bool BF16C = false>
 cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool pdl,
                         const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st,
                         bool* fits) {
-    auto kern = decode_kernel<MODE, BIG, EARLY>;
+    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C>;
     static bool configured = false;   // attributes are per function, set once
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1008,32 +1029,29 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
         if (smem > 227 * 1024) return cudaErrorInvalidValue;
         bool fits = false;
         const bool early = early_prefetch && mode == kModeFull;
-        switch (mode * 4 + (big ? 2 : 0) + (early ? 1 : 0)) {
-            case kModeSelect * 4:
-                e = launch_mode<kModeSelect, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            case kModeSelect * 4 + 2:
-                e = launch_mode<kModeSelect, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            case kModeAttend * 4:
-                e = launch_mode<kModeAttend, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            case kModeAttend * 4 + 2:
-                e = launch_mode<kModeAttend, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            case kModeFull * 4:
-                e = launch_mode<kModeFull, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            case kModeFull * 4 + 1:
-                e = launch_mode<kModeFull, false, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            case kModeFull * 4 + 2:
-                e = launch_mode<kModeFull, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
-            default:
-                e = launch_mode<kModeFull, true, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
-                break;
+#define ABSP_LAUNCH(M, B, E, F) \
+    launch_mode<M, B, E, F>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits)
+        const bool bf = a.cfmt == ABSP_CENTROIDS_BF16;
+        if (mode == kModeAttend) {
+            e = big ? ABSP_LAUNCH(kModeAttend, true, false, false)
+                    : ABSP_LAUNCH(kModeAttend, false, false, false);
+        } else if (mode == kModeSelect) {
+            if (big) e = bf ? ABSP_LAUNCH(kModeSelect, true, false, true)
+                            : ABSP_LAUNCH(kModeSelect, true, false, false);
+            else e = bf ? ABSP_LAUNCH(kModeSelect, false, false, true)
+                        : ABSP_LAUNCH(kModeSelect, false, false, false);
+        } else if (big) {
+            if (early) e = bf ? ABSP_LAUNCH(kModeFull, true, true, true)
+                              : ABSP_LAUNCH(kModeFull, true, true, false);
+            else e = bf ? ABSP_LAUNCH(kModeFull, true, false, true)
+                        : ABSP_LAUNCH(kModeFull, true, false, false);
+        } else {
+            if (early) e = bf ? ABSP_LAUNCH(kModeFull, false, true, true)
+                              : ABSP_LAUNCH(kModeFull, false, true, false);
+            else e = bf ? ABSP_LAUNCH(kModeFull, false, false, true)
+                        : ABSP_LAUNCH(kModeFull, false, false, false);
         }
+#undef ABSP_LAUNCH
         if (e != cudaSuccess || fits) return e;
         // this cluster shape cannot be resident: retry with a smaller one
     }

@@ -69,7 +69,8 @@ extern "C" absp_status absp_build_quantize_noalloc(const absp_layer_kv* kv,
     if (cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return ABSP_ERR_CUDA;
     const absp::BuildWs w = absp::build_ws_layout(ws, d);
     if (absp::launch_build(d, w, s) != cudaSuccess) return ABSP_ERR_CUDA;
-    if (absp::launch_quantize(d, w, out->codes, out->scale, out->zp, s) != cudaSuccess)
+    if (absp::launch_quantize(d, w, out->codes, out->scale, out->zp, out->format, s) !=
+        cudaSuccess)
         return ABSP_ERR_CUDA;
     if (device_status != nullptr &&
         cudaMemcpyAsync(device_status, ws, 2 * sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=

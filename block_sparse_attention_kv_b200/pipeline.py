@@ -13,7 +13,8 @@ from . import abi
 
 
 class DeviceLayer:
-    def __init__(self, data, budget: int = None, stream=None, block_size=None):
+    def __init__(self, data, budget: int = None, stream=None, block_size=None,
+                 fmt: int = abi.ABSP_CENTROIDS_INT4):
         """`data` is a synth.LayerData on a CUDA device; `block_size`
         overrides its per-KV-head block-size table (same cache, other
         blocking)."""
@@ -23,7 +24,7 @@ class DeviceLayer:
         self.block_size = list(data.block_size if block_size is None else block_size)
         self.kv = abi.LayerKV(data.seq_lens, data.page_table, data.k_pages, data.v_pages,
                               self.block_size, data.num_q_heads)
-        self.cent = abi.alloc_centroids(self.kv, self.device)
+        self.cent = abi.alloc_centroids(self.kv, self.device, fmt)
         self.build_ws = None
         dws = abi.absp_decode_workspace_size(self.kv, self.budget)
         self.ws = abi.alloc_workspace(dws, self.device)
@@ -76,9 +77,11 @@ class DeviceLayer:
 
     # -- views of the centroid store ----------------------------------------
     def codes_of(self, s: int, h: int, n: int) -> torch.Tensor:
-        """Packed code rows [n][64] of (sequence s, KV head h)."""
+        """Centroid rows of (sequence s, KV head h): [n][64] packed INT4
+        codes, or [n][256] bytes of bf16 centroids."""
+        rb = 256 if self.cent.format == abi.ABSP_CENTROIDS_BF16 else 64
         r0 = abi.absp_centroid_row_offset(self.kv, s, h)
-        return self.cent.codes[r0 * 64:(r0 + n) * 64].view(n, 64)
+        return self.cent.codes[r0 * rb:(r0 + n) * rb].view(n, rb)
 
     def params_of(self, s: int, h: int):
         Hkv = self.data.num_kv_heads

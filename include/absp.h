@@ -93,7 +93,18 @@ typedef struct absp_centroids {
     uint8_t* codes;              /* device, 256-byte aligned               */
     float* scale;                /* device [S][Hkv][128]                   */
     int32_t* zp;                 /* device [S][Hkv][128]                   */
+    int32_t format;              /* ABSP_CENTROIDS_INT4 (0) or _BF16 (1)   */
 } absp_centroids;
+
+/* Centroid storage formats (the precision comparison of Fig. 13: INT4
+ * codes vs unquantised BF16 centroids).
+ *   ABSP_CENTROIDS_INT4: as above, 64-byte rows of packed nibbles plus
+ *     per-channel scale / zp.
+ *   ABSP_CENTROIDS_BF16: 256-byte rows, channel c as the bf16 nearest to
+ *     the fp64 mean (ties to even, no intermediate rounding); scale and zp
+ *     are neither read nor written (may be NULL). */
+#define ABSP_CENTROIDS_INT4 0
+#define ABSP_CENTROIDS_BF16 1
 
 /* Human-readable name of a status code (static string, never NULL). */
 ABSP_API const char* absp_status_string(absp_status status);
@@ -102,7 +113,14 @@ ABSP_API const char* absp_status_string(absp_status status);
 ABSP_API absp_status absp_centroid_sizes(const absp_layer_kv* kv, size_t* codes_bytes,
                                 size_t* scale_bytes, size_t* zp_bytes);
 
-/* First code row of (seq, kv_head) in absp_centroids.codes (host only). */
+/* Bytes of the centroid buffers for a given format (ABSP_CENTROIDS_*);
+ * scale / zp bytes are 0 for ABSP_CENTROIDS_BF16. */
+ABSP_API absp_status absp_centroid_sizes_fmt(const absp_layer_kv* kv, int32_t format,
+                                             size_t* codes_bytes, size_t* scale_bytes,
+                                             size_t* zp_bytes);
+
+/* First code row of (seq, kv_head) in absp_centroids.codes (host only);
+ * rows are 64 bytes (INT4) or 256 bytes (BF16). */
 ABSP_API absp_status absp_centroid_row_offset(const absp_layer_kv* kv, int32_t seq,
                                      int32_t kv_head, int64_t* row);
 
@@ -138,7 +156,9 @@ ABSP_API absp_status absp_build_centroids(const absp_layer_kv* kv, void* ws,
  *   scale = fp32((max - min) / 15), zp = rint(-min / scale) (int32, not
  *   clamped to 4 bits), code = clamp(rint(c / scale) + zp, 0, 15),
  * rint = round half to even, all in fp64 except the stored scale; a channel
- * with max == min gets scale 0, zp 0, codes 0.  Writes `out`. */
+ * with max == min gets scale 0, zp 0, codes 0.  Writes `out`.  With
+ * out->format == ABSP_CENTROIDS_BF16 it writes the bf16-rounded centroids
+ * instead (no quantisation). */
 ABSP_API absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws,
                                     size_t ws_bytes, const absp_centroids* out,
                                     void* stream);
@@ -146,7 +166,8 @@ ABSP_API absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws,
 /* Steps 3-4 (Fig. 1 "dot product estimation", "importance score",
  * "top-K selection"): for every (seq, kv_head), qbar = sum of the GQA
  * group's queries (q: device bf16 [S][Hq][128]), score[b] =
- * sum_ch qbar[ch] * (code[b][ch] - zp[ch]) * scale[ch] (fp32), then the
+ * sum_ch qbar[ch] * (code[b][ch] - zp[ch]) * scale[ch] (fp32; with BF16
+ * centroids sum_ch qbar[ch] * centroid[b][ch]), then the
  * K_h = min(n_h, max(1, budget / bs_h)) highest scores, ties to the lower
  * block index.  Writes sel[(s*Hkv + h) * kmax + i], i < K_h, ascending
  * block indices (kmax from absp_select_capacity), and sel_count[s*Hkv + h]

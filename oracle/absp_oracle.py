@@ -153,6 +153,26 @@ def dequantize(qc: QuantizedCentroids) -> np.ndarray:
         * qc.scale.astype(np.float64)[None, :]
 
 
+def round_bf16(x) -> np.ndarray:
+    """fp64 -> nearest bf16 value (ties to even), returned as fp64.
+
+    A bf16 number has 8 significant bits and the exponent range of fp32:
+    with x = m * 2**e, 0.5 <= |m| < 1, its spacing near x is 2**(e - 8)
+    (2**-133 below the smallest normal 2**-126).  Rounding to a multiple of
+    that spacing, ties to even, is exact in fp64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    q = np.ldexp(1.0, np.maximum(e, -125) - 8)
+    return np.rint(x / q) * q
+
+
+def bf16_bits_of(x) -> np.ndarray:
+    """Bit patterns (uint16) of values that are exactly bf16."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
 def pack_codes(codes: np.ndarray) -> np.ndarray:
     """[n][128] nibbles -> [n][64] bytes; channel 2i in the low nibble."""
     c = np.asarray(codes, dtype=np.uint8)
@@ -271,14 +291,15 @@ def decode_head(q_heads: np.ndarray, kv_head: int, group: int, chat: np.ndarray,
     return sc, k, sel, outs
 
 
-def run_layer(layer, quantize: bool = True, sel_override=None,
+def run_layer(layer, quantize=True, sel_override=None,
               heads=None, with_attention: bool = True) -> LayerResult:
     """All five steps for every (sequence, KV head) of a host layer.
 
     `layer` carries q_bits [S][Hq][128], k_bits / v_bits
     [P][Hkv][16][128] (uint16 bf16 bits), page_table [S][max_pages],
     seq_lens [S], block_size [Hkv] and budget.  `quantize=False` scores the
-    fp64 centroids directly (the unquantised variant).  `sel_override`
+    fp64 centroids directly (the unquantised variant); `quantize="bf16"`
+    scores the centroids rounded to bf16 (the BF16-centroid variant).  `sel_override`
     maps (s, h) -> block list to attend over instead of the oracle's own
     selection.  `heads` restricts the work to some (s, h) pairs.
     """
@@ -296,7 +317,10 @@ def run_layer(layer, quantize: bool = True, sel_override=None,
             keys, vals = head_keys_values(layer, s, h)
             cent = build_centroids(keys, bs)
             qc = quantize_centroids(cent)
-            chat = dequantize(qc) if quantize else cent
+            if quantize == "bf16":
+                chat = round_bf16(cent)
+            else:
+                chat = dequantize(qc) if quantize else cent
             ov = None if sel_override is None else sel_override[(s, h)]
             sc, k, sel, outs = decode_head(qf, h, G, chat, keys, vals, bs, L,
                                            layer.budget, sel_override=ov)

@@ -62,6 +62,18 @@ def compare_codes(rep: Report, hr: O.HeadResult, packed_gpu: np.ndarray,
         rep.notes.append(f"codes differ in {bad} bytes")
 
 
+def compare_bf16_centroids(rep: Report, hr: O.HeadResult, rows_gpu: np.ndarray) -> None:
+    """BF16 centroid rows (256 bytes each) against the oracle's rounding."""
+    n = hr.centroids.shape[0]
+    want = O.bf16_bits_of(O.round_bf16(hr.centroids))
+    got = np.ascontiguousarray(np.asarray(rows_gpu, dtype=np.uint8).reshape(n, 256)) \
+        .view(np.uint16).reshape(n, 128)
+    bad = int(np.count_nonzero(got != want))
+    rep.code_mismatch += bad
+    if bad:
+        rep.notes.append(f"bf16 centroids differ in {bad} channels")
+
+
 def compare_selection(rep: Report, hr: O.HeadResult, sel_gpu) -> None:
     got = [int(x) for x in sel_gpu]
     want = hr.sel.tolist()

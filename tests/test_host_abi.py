@@ -76,6 +76,10 @@ def test_sizes_follow_the_layout(abi):
     assert abi.absp_select_capacity(kv, 40) == 2          # max(1, 40/16)
     ws = abi.absp_build_workspace_size(kv)
     assert ws == 256 + 2 * 2 * 128 * 8 + 640 * 128 * 8
+    assert abi.absp_centroid_sizes_fmt(kv, abi.ABSP_CENTROIDS_INT4) == (codes, scale, zp)
+    assert abi.absp_centroid_sizes_fmt(kv, abi.ABSP_CENTROIDS_BF16) == (640 * 256, 0, 0)
+    with pytest.raises(abi.AbspError):
+        abi.absp_centroid_sizes_fmt(kv, 7)
 
 
 @pytest.mark.parametrize("over,status", [

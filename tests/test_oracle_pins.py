@@ -167,6 +167,26 @@ def test_pack_nibble_order_round_trip():
     assert np.array_equal(O.unpack_codes(p), codes)
 
 
+def test_round_bf16_matches_torch_on_fp32_inputs():
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal(5000) * 10.0 ** rng.integers(-30, 30, 5000),
+                        [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0]])
+    x32 = x.astype(np.float32)
+    want = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x32.astype(np.float64)), want)
+
+
+def test_round_bf16_has_no_double_rounding():
+    # halfway between 1 and 1+2^-7 plus a tail that fp32 cannot hold: the
+    # correct result rounds up; rounding through fp32 first would tie to 1.0
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -40
+    assert O.round_bf16(x) == 1.0 + 2.0 ** -7
+    assert O.round_bf16(1.0 + 2.0 ** -8) == 1.0            # exact tie -> even
+    assert O.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert O.round_bf16(2.0 ** -133 * 0.75) == 2.0 ** -133  # subnormal spacing
+    assert O.bf16_bits_of(np.array([1.0, -2.0]))[1] == 0xC000
+
+
 # ------------------------------------------------------- step 3: scores --
 
 def test_group_query_and_score_equal_sum_of_per_head_dots():

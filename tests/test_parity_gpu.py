@@ -32,12 +32,13 @@ def _bits(t):
     return t.contiguous().view(torch.int16)
 
 
-def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None):
+def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None, fmt=0):
     abi, pipeline = lib
     d = data if data is not None else synth.make_layer(w, layer, "cuda")
     if modify is not None:
         modify(d)
-    dl = pipeline.DeviceLayer(d, budget)
+    dl = pipeline.DeviceLayer(d, budget, fmt=fmt)
+    bf16 = fmt == abi.ABSP_CENTROIDS_BF16
     dl.build_centroids()
     dl.score_select()
     dl.sparse_decode()
@@ -61,16 +62,20 @@ def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None):
     sel = dl.sel.cpu().numpy()
     cnt = dl.sel_count.cpu().numpy()
     override = {(i, h): sel[s, h, :cnt[s, h]] for i, s in enumerate(seqs) for h in range(Hkv)}
-    res = O.run_layer(hl, sel_override=override)
+    res = O.run_layer(hl, quantize="bf16" if bf16 else True, sel_override=override)
     rep = PR.Report()
     for i, s in enumerate(seqs):
         for h in range(Hkv):
             hr = res.heads[(i, h)]
             rep.heads += 1
             n = hr.centroids.shape[0]
-            scale, zp = dl.params_of(s, h)
-            packed = dl.codes_of(s, h, n).cpu().numpy() if n else np.zeros((0, 64), np.uint8)
-            PR.compare_codes(rep, hr, packed, scale.cpu().numpy(), zp.cpu().numpy())
+            if bf16:
+                rows = dl.codes_of(s, h, n).cpu().numpy() if n else np.zeros((0, 256), np.uint8)
+                PR.compare_bf16_centroids(rep, hr, rows)
+            else:
+                scale, zp = dl.params_of(s, h)
+                packed = dl.codes_of(s, h, n).cpu().numpy() if n else np.zeros((0, 64), np.uint8)
+                PR.compare_codes(rep, hr, packed, scale.cpu().numpy(), zp.cpu().numpy())
             PR.compare_selection(rep, hr, sel[s, h, :cnt[s, h]])
     outg = out_split[torch.as_tensor(seqs, device=out_split.device)].float().cpu().numpy()
     PR.compare_outputs(rep, outg, res.out)
@@ -160,6 +165,24 @@ def test_outlier_block_forces_radix_fallback(lib):
         ids = d.page_table[0, 5:6].long()                 # block 5 of head 0 (bs 16)
         d.k_pages[ids, 0] = (d.k_pages[ids, 0].float() * 4096.0).to(torch.bfloat16)
     run_case(lib, w, modify=modify)
+
+
+# ----------------------------------------------- BF16 centroid variant --
+
+def test_bf16_centroids_tiny(lib):
+    abi, _ = lib
+    run_case(lib, synth.WORKLOADS["tiny_8k"], fmt=abi.ABSP_CENTROIDS_BF16)
+
+
+def test_bf16_centroids_ragged_gqa16(lib):
+    abi, _ = lib
+    w = synth.custom("bf16_ragged", 3, 32, 2, [3000, 77, 1025], [32, 16], 384, seed=60)
+    run_case(lib, w, fmt=abi.ABSP_CENTROIDS_BF16)
+
+
+def test_bf16_centroids_llama31_8b_32k(lib):
+    abi, _ = lib
+    run_case(lib, synth.WORKLOADS["llama31_8b_32k"], fmt=abi.ABSP_CENTROIDS_BF16)
 
 
 def test_host_buffers_match_device_step(lib):
