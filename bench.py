@@ -413,6 +413,25 @@ def gpu_arm(args):
         x.check()
     del g_plain
 
+    # incremental tail-row update (one launch per layer); with unchanged
+    # lengths it rewrites every tail row with the same bytes
+    append = None
+    if not args.no_variants:
+        ga = torch.cuda.CUDAGraph()
+        for x in layers:
+            abi.absp_append_centroids(x.kv, x.cent, None, x.ws, sc)
+        stream.synchronize()
+        with torch.cuda.graph(ga, stream=stream):
+            for x in layers:
+                abi.absp_append_centroids(x.kv, x.cent, None, x.ws, sc)
+        with torch.cuda.stream(stream):
+            ms_a = timed(ga, args.steps, args.warmup)
+        for x in layers:
+            x.check()
+        append = {"us_per_layer": ms_a / (args.steps * L) * 1e3,
+                  "note": "absp_append_centroids, all 8 KV heads of one layer per launch"}
+        del ga
+
     # fixed block size for every KV head (the uniform-block methods the page
     # compares against) and unquantised bf16 centroids (its precision
     # baseline), on the same caches, queries and token budget
@@ -423,9 +442,10 @@ def gpu_arm(args):
                           layers[0].data.k_pages, layers[0].data.v_pages,
                           [16] * layers[0].data.num_kv_heads, layers[0].data.num_q_heads)
         fws = abi.alloc_workspace(abi.absp_build_workspace_size(big), dev)
-        cases = [(f"fixed_block_{b}", b, abi.ABSP_CENTROIDS_INT4) for b in (16, 32, 64)]
-        cases.append(("bf16_centroids", None, abi.ABSP_CENTROIDS_BF16))
-        for name, bsz, fmt in cases:
+        cases = [(f"fixed_block_{b}", b, abi.ABSP_CENTROIDS_INT4, 0) for b in (16, 32, 64)]
+        cases.append(("bf16_centroids", None, abi.ABSP_CENTROIDS_BF16, 0))
+        cases.append(("group_max", None, abi.ABSP_CENTROIDS_INT4, abi.ABSP_STEP_GROUP_MAX))
+        for name, bsz, fmt, vflags in cases:
             vl = [pipeline.DeviceLayer(
                 x.data, stream=sc, fmt=fmt,
                 block_size=None if bsz is None else [bsz] * x.data.num_kv_heads)
@@ -434,17 +454,18 @@ def gpu_arm(args):
             for y in vl:
                 abi.absp_build_centroids(y.kv, fws, sc)
                 abi.absp_quantize_centroids(y.kv, fws, y.cent, sc)
-                y.score_select()
+                y.score_select(flags=vflags)
                 stream.synchronize()
                 vb.append(step_bytes(y.data, y.sel.cpu().numpy(), y.sel_count.cpu().numpy(),
                                      y.block_size, fmt == abi.ABSP_CENTROIDS_BF16))
-                abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws, EARLY, sc)
+                abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws,
+                                        EARLY | vflags, sc)
             stream.synchronize()
             gv = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gv, stream=stream):
                 for y in vl:
                     abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws,
-                                            EARLY, sc)
+                                            EARLY | vflags, sc)
             with torch.cuda.stream(stream):
                 ms_v = timed(gv, args.steps, args.warmup)
             for y in vl:
@@ -528,6 +549,7 @@ def gpu_arm(args):
                                "ms_per_step": ms_plain / args.steps,
                                "note": "absp_decode_step, no reads before the previous "
                                        "launch completes"}},
+        "append": append,
         "clocks": clocks,
         "rebuild": {"ms_per_layer": rebuild_ms, "bytes_per_layer": rb_bytes,
                     "achieved_gbs": rb_bytes / (rebuild_ms * 1e-3) / 1e9,

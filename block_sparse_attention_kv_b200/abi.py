@@ -27,6 +27,7 @@ ABSP_ERR_DEVICE_FAULT = 4
 ABSP_ERR_TIMEOUT = 5
 
 ABSP_STEP_EARLY_PREFETCH = 1
+ABSP_STEP_GROUP_MAX = 2
 ABSP_CENTROIDS_INT4 = 0
 ABSP_CENTROIDS_BF16 = 1
 
@@ -90,6 +91,11 @@ def _load() -> ctypes.CDLL:
                                          P(absp_centroids), c_void_p]),
         "absp_score_select": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
                                    c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+        "absp_append_centroids": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_void_p,
+                                       c_size_t, c_void_p]),
+        "absp_score_select_ex": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
+                                      c_void_p, c_void_p, c_void_p, c_size_t, c_uint32,
+                                      c_void_p]),
         "absp_sparse_decode": (st, [P(absp_layer_kv), c_void_p, c_void_p, c_void_p, c_int32,
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
         "absp_decode_step": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
@@ -114,7 +120,9 @@ EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_sizes_fm
             "absp_centroid_row_offset",
             "absp_build_workspace_size", "absp_decode_workspace_size",
             "absp_select_capacity", "absp_workspace_init", "absp_build_centroids",
-            "absp_quantize_centroids", "absp_score_select", "absp_sparse_decode",
+            "absp_quantize_centroids", "absp_append_centroids", "absp_score_select",
+            "absp_score_select_ex",
+            "absp_sparse_decode",
             "absp_decode_step", "absp_decode_step_ex", "absp_decode_step_host",
             "absp_check_device_error", "absp_build_quantize_noalloc")
 
@@ -280,6 +288,20 @@ def absp_score_select(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int
     _check(_lib.absp_score_select(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(sel),
                                   _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
            "absp_score_select")
+
+
+def absp_append_centroids(kv: LayerKV, cent: Centroids, exceeded, ws: torch.Tensor,
+                          stream=None) -> None:
+    _check(_lib.absp_append_centroids(kv.ref, cent.ref, _ptr(exceeded), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "absp_append_centroids")
+
+
+def absp_score_select_ex(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
+                         sel: torch.Tensor, sel_count: torch.Tensor, ws: torch.Tensor,
+                         flags: int, stream=None) -> None:
+    _check(_lib.absp_score_select_ex(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(sel),
+                                     _ptr(sel_count), _ptr(ws), ws.numel(), int(flags),
+                                     _stream(stream)), "absp_score_select_ex")
 
 
 def absp_sparse_decode(kv: LayerKV, q: torch.Tensor, sel: torch.Tensor,

@@ -184,6 +184,7 @@ absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* 
     a.scale = cent ? cent->scale : nullptr;
     a.zp = cent ? cent->zp : nullptr;
     a.cfmt = cent ? cent->format : ABSP_CENTROIDS_INT4;
+    a.group_max = (flags & ABSP_STEP_GROUP_MAX) != 0 ? 1 : 0;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.out = static_cast<__nv_bfloat16*>(out);
     a.sel = sel;
@@ -305,6 +306,18 @@ absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws, size_t ws
                                      out->format, static_cast<cudaStream_t>(stream)));
 }
 
+absp_status absp_append_centroids(const absp_layer_kv* kv, const absp_centroids* cent,
+                                  int32_t* exceeded, void* ws, size_t ws_bytes, void* stream) {
+    KvDesc d;
+    absp_status st = make_desc(kv, &d, false);
+    if (st != ABSP_OK) return st;
+    if ((st = check_cent(cent)) != ABSP_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, kWsHeader)) != ABSP_OK) return st;
+    if (exceeded != nullptr && !aligned(exceeded, 4)) return ABSP_ERR_INVALID_ARG;
+    return from_cuda(launch_append(d, cent->codes, cent->scale, cent->zp, cent->format, exceeded,
+                                   static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
 absp_status absp_score_select(const absp_layer_kv* kv, const absp_centroids* cent, const void* q,
                               int32_t budget_tokens, int32_t* sel, int32_t* sel_count, void* ws,
                               size_t ws_bytes, void* stream) {
@@ -329,9 +342,18 @@ absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centroids* cent
 absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                 const void* q, int32_t budget_tokens, void* out, void* ws,
                                 size_t ws_bytes, uint32_t flags, void* stream) {
-    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH)) != 0) return ABSP_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX)) != 0)
+        return ABSP_ERR_INVALID_ARG;
     return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
                       stream, flags);
+}
+
+absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* cent, const void* q,
+                                 int32_t budget_tokens, int32_t* sel, int32_t* sel_count,
+                                 void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
+    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_GROUP_MAX)) != 0) return ABSP_ERR_INVALID_ARG;
+    return run_decode(kModeSelect, kv, cent, q, budget_tokens, sel, sel_count, nullptr, ws,
+                      ws_bytes, stream, flags);
 }
 
 absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids* cent,

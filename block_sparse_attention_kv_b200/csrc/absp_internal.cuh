@@ -293,6 +293,10 @@ cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st);
 cudaError_t launch_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
                             int32_t* zp, int format, cudaStream_t st);
 
+// Incremental tail-row update after appended tokens (centroids.cu)
+cudaError_t launch_append(const KvDesc& kv, uint8_t* codes, const float* scale, const int32_t* zp,
+                          int format, int32_t* exceeded, int32_t* err, cudaStream_t st);
+
 // Decode steps (decode.cu)
 enum DecodeMode : int { kModeSelect = 1, kModeAttend = 2, kModeFull = 3 };
 
@@ -310,6 +314,7 @@ struct DecodeArgs {
     int32_t* err;
     int32_t nmax;                 // bound on blocks per head for this layer
     int32_t cfmt;                 // centroid format (ABSP_CENTROIDS_*)
+    int32_t group_max;            // score = max over the GQA group's heads
 };
 // early_prefetch: codes, parameters, lengths and page table are read before
 // the programmatic-dependency wait (only the query after it).

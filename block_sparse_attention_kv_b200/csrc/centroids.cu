@@ -249,6 +249,75 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
     }
 }
 
+// Incremental update after tokens were appended: one warp per
+// (sequence, KV head) recomputes the centroid of the block that holds the
+// last token (token-order fp64 sum over that block's keys) and stores it
+// under the existing per-channel parameters (INT4, clamped) or as bf16.
+// exceeded[s][h] counts INT4 channels whose unclamped code left 0..15.
+__global__ void __launch_bounds__(kBuildWarps * 32)
+    centroid_append_kernel(const KvDesc kv, uint8_t* __restrict__ codes,
+                           const float* __restrict__ scale, const int32_t* __restrict__ zp,
+                           int format, int32_t* __restrict__ exceeded, int32_t* err) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = blockIdx.x * kBuildWarps + warp;
+    if (pair >= kv.S * kv.Hkv) return;
+    const int s = pair / kv.Hkv, h = pair % kv.Hkv;
+    int len = kv.seq_lens[s];
+    if (len < 0 || len > kv.max_pages * kPage) {
+        if (lane == 0 && h == 0) set_error(err, ABSP_ERR_DEVICE_FAULT, s);
+        len = 0;
+    }
+    int count = 0;
+    if (len > 0) {
+        const int bs = kv.bs[h];
+        const int b = (len - 1) / bs;
+        const int t0 = b * bs;
+        const int32_t* pt = kv.page_table + static_cast<int64_t>(s) * kv.max_pages;
+        double a[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int t = t0; t < len; ++t) {
+            const int phys = pt[t / kPage];
+            if (phys < 0 || phys >= kv.num_phys_pages) {
+                if (lane == 0) set_error(err, ABSP_ERR_DEVICE_FAULT, s);
+                continue;
+            }
+            const uint2 v = ld_nc_u2(kv.k_pages +
+                                     ((static_cast<int64_t>(phys) * kv.Hkv + h) * kPage + t % kPage) * kD +
+                                     lane * 4);
+            a[0] += static_cast<double>(bf16lo(v.x));
+            a[1] += static_cast<double>(bf16hi(v.x));
+            a[2] += static_cast<double>(bf16lo(v.y));
+            a[3] += static_cast<double>(bf16hi(v.y));
+        }
+        const double cnt = static_cast<double>(len - t0);
+        const int64_t row = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h] + b;
+        if (format == ABSP_CENTROIDS_BF16) {
+            uint2 o;
+            o.x = f64_to_bf16_rne(a[0] / cnt) | (f64_to_bf16_rne(a[1] / cnt) << 16);
+            o.y = f64_to_bf16_rne(a[2] / cnt) | (f64_to_bf16_rne(a[3] / cnt) << 16);
+            *reinterpret_cast<uint2*>(codes + row * (2 * kD) + lane * 8) = o;
+        } else {
+            const int64_t pi = (static_cast<int64_t>(s) * kv.Hkv + h) * kD + lane * 4;
+            uint32_t packed = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const double sc = static_cast<double>(scale[pi + i]);
+                uint32_t code = 0;
+                if (sc > 0.0) {
+                    const double qv = rint((a[i] / cnt) / sc) + static_cast<double>(zp[pi + i]);
+                    if (qv < 0.0 || qv > 15.0) ++count;
+                    code = static_cast<uint32_t>(fmin(fmax(qv, 0.0), 15.0));
+                }
+                packed |= code << (4 * i);
+            }
+            *reinterpret_cast<uint16_t*>(codes + row * kRowBytes + lane * 2) =
+                static_cast<uint16_t>(packed);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) count += __shfl_xor_sync(0xffffffffu, count, o);
+    if (exceeded != nullptr && lane == 0) exceeded[pair] = count;
+}
+
 }  // namespace
 
 size_t build_ws_bytes(const KvDesc& kv) {
@@ -281,6 +350,14 @@ cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st) {
     e = cudaMemsetAsync(w.minmax + pairs, 0, pairs * sizeof(unsigned long long), st);
     if (e != cudaSuccess) return e;
     centroid_build_kernel<<<chunk_grid(kv), kBuildWarps * 32, 0, st>>>(kv, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append(const KvDesc& kv, uint8_t* codes, const float* scale, const int32_t* zp,
+                          int format, int32_t* exceeded, int32_t* err, cudaStream_t st) {
+    const int pairs = kv.S * kv.Hkv;
+    centroid_append_kernel<<<(pairs + kBuildWarps - 1) / kBuildWarps, kBuildWarps * 32, 0, st>>>(
+        kv, codes, scale, zp, format, exceeded, err);
     return cudaGetLastError();
 }
 

@@ -72,7 +72,13 @@ struct Params {
     uint32_t small_off;
     uint32_t scratch_off;         // select scratch inside region B
     int32_t slots;                // page buffers per warp (1 or 2)
+    int32_t group_max;            // score = max over the group's heads
+    uint32_t wg_off;              // per-head weights inside region B
 };
+
+// per-head score weights for the group-max variant: [G][8 lanes][20]
+// floats (16 used), padded so the 8 lanes of a row read distinct banks
+constexpr int kWgStride = 160;
 
 struct Small {                    // fixed-size shared scratch
     unsigned long long bar_code[kStages];
@@ -462,6 +468,14 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             for (int j = 0; j < G; ++j) qb += __bfloat162float(qh[j * kD]);
             sm.w[tid] = BF16C ? qb : qb * scl;
             sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
+            if (p.group_max) {
+                float* wg = reinterpret_cast<float*>(regB + p.wg_off);
+                const int slot = (tid >> 4) * 20 + (tid & 15);
+                for (int j = 0; j < G; ++j) {
+                    const float qj = __bfloat162float(qh[j * kD]);
+                    wg[j * kWgStride + slot] = BF16C ? qj : qj * scl;
+                }
+            }
         }
         __syncthreads();
         const int sub = tid & 7, grp = tid >> 3;  // 32 groups of 8 lanes
@@ -493,39 +507,87 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                 for (int u = 0; u < 4; ++u) {
                     const int r = r4 + u;
                     float acc = 0.0f;
-                    if constexpr (BF16C) {
-                        // 16 bf16 centroid channels per lane: score += qbar * c
-                        uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
-                        if (r < rows) {
-                            const uint4* src = reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
-                            y0 = src[0];
-                            y1 = src[1];
-                        }
-                        const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                    if (!p.group_max) {
+                        if constexpr (BF16C) {
+                            // 16 bf16 centroid channels per lane: score += qbar * c
+                            uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
+                            if (r < rows) {
+                                const uint4* src = reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
+                                y0 = src[0];
+                                y1 = src[1];
+                            }
+                            const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            acc = fmaf(wr[2 * k], bf16lo(yy[k]), acc);
-                            acc = fmaf(wr[2 * k + 1], bf16hi(yy[k]), acc);
+                            for (int k = 0; k < 8; ++k) {
+                                acc = fmaf(wr[2 * k], bf16lo(yy[k]), acc);
+                                acc = fmaf(wr[2 * k + 1], bf16hi(yy[k]), acc);
+                            }
+                        } else {
+                            uint2 x = make_uint2(0u, 0u);
+                            if (r < rows) x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const float f =
+                                    __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
+                                acc = fmaf(wr[k], f, acc);
+                            }
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const float f =
+                                    __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
+                                acc = fmaf(wr[8 + k], f, acc);
+                            }
                         }
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
                     } else {
-                        uint2 x = make_uint2(0u, 0u);
-                        if (r < rows) x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
+                        // variant: the largest of the group's per-head scores
+                        float f[16];
+                        if constexpr (BF16C) {
+                            uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
+                            if (r < rows) {
+                                const uint4* src =
+                                    reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
+                                y0 = src[0];
+                                y1 = src[1];
+                            }
+                            const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const float f =
-                                __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
-                            acc = fmaf(wr[k], f, acc);
+                            for (int k = 0; k < 8; ++k) {
+                                f[2 * k] = bf16lo(yy[k]);
+                                f[2 * k + 1] = bf16hi(yy[k]);
+                            }
+                        } else {
+                            uint2 x = make_uint2(0u, 0u);
+                            if (r < rows)
+                                x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                f[k] = __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
+                                f[8 + k] =
+                                    __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
+                            }
                         }
+                        const float* wg = reinterpret_cast<const float*>(regB + p.wg_off) + sub * 20;
+                        acc = -INFINITY;
+                        for (int jh = 0; jh < G; ++jh) {
+                            const float4* w4 = reinterpret_cast<const float4*>(wg + jh * kWgStride);
+                            float a = 0.0f;
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const float f =
-                                __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
-                            acc = fmaf(wr[8 + k], f, acc);
+                            for (int k4 = 0; k4 < 4; ++k4) {
+                                const float4 wv = w4[k4];
+                                a = fmaf(wv.x, f[4 * k4], a);
+                                a = fmaf(wv.y, f[4 * k4 + 1], a);
+                                a = fmaf(wv.z, f[4 * k4 + 2], a);
+                                a = fmaf(wv.w, f[4 * k4 + 3], a);
+                            }
+                            a += __shfl_xor_sync(0xffffffffu, a, 1);
+                            a += __shfl_xor_sync(0xffffffffu, a, 2);
+                            a += __shfl_xor_sync(0xffffffffu, a, 4);
+                            acc = fmaxf(acc, a);
                         }
                     }
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
                     q4[u] = r < rows ? acc : 0.0f;
                     if (r < rows) {
                         lmin = fminf(lmin, acc);
@@ -997,6 +1059,8 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     prm.budget = a.budget;
     prm.err = a.err;
     prm.qk_scale_log2 = kLog2e / sqrtf(static_cast<float>(kD));
+    prm.group_max = a.group_max;
+    prm.wg_off = 0;
 
     int C = pick_cluster(pairs, num_sms);
     cudaError_t e = cudaSuccess;
@@ -1008,7 +1072,9 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
         if (do_select) {
             // score slots for every row, rounded up to whole groups of 4
             scratch = (static_cast<size_t>(a.nmax + 3) / 4) * 16;
-            regB = std::max(regB, scratch + kSelectScratch);
+            prm.wg_off = static_cast<uint32_t>(scratch + kSelectScratch);
+            regB = std::max(regB, scratch + kSelectScratch +
+                                      (a.group_max ? static_cast<size_t>(G) * kWgStride * 4 : 0));
             regA = std::max(regA, static_cast<size_t>(kStages) * kStageBytes);
         }
         if (do_attend) {

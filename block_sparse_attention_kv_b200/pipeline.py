@@ -47,9 +47,14 @@ class DeviceLayer:
             self.build_ws = None
 
     # -- steps 3-5 --------------------------------------------------------
-    def score_select(self, q=None):
-        abi.absp_score_select(self.kv, self.cent, self.data.q if q is None else q,
-                              self.budget, self.sel, self.sel_count, self.ws, self.stream)
+    def score_select(self, q=None, flags: int = 0):
+        q = self.data.q if q is None else q
+        if flags:
+            abi.absp_score_select_ex(self.kv, self.cent, q, self.budget, self.sel,
+                                     self.sel_count, self.ws, flags, self.stream)
+        else:
+            abi.absp_score_select(self.kv, self.cent, q, self.budget, self.sel,
+                                  self.sel_count, self.ws, self.stream)
 
     def sparse_decode(self, q=None, out=None):
         abi.absp_sparse_decode(self.kv, self.data.q if q is None else q, self.sel,

@@ -163,6 +163,22 @@ ABSP_API absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws,
                                     size_t ws_bytes, const absp_centroids* out,
                                     void* stream);
 
+/* Incremental update during decode (Fig. 5: block sizes are fixed, so the
+ * store is kept up to date instead of rebuilt).  Call after the caller has
+ * written the new tokens' K/V into the pages and raised seq_lens.  For every
+ * (seq, kv_head) the centroid of the block holding the last token is
+ * recomputed from that block's keys (token-order fp64 mean, the value a
+ * full rebuild gives) and stored under the EXISTING per-channel scale / zp
+ * (INT4: code = clamp(rint(c/scale) + zp, 0, 15)) or as bf16 (BF16 format).
+ * The per-channel parameters are not changed.  exceeded (optional, device
+ * int32 [S][Hkv]) receives, per (seq, head), the number of channels whose
+ * unclamped code left 0..15 (channels with scale 0 are not counted): a
+ * non-zero count means the parameters no longer cover the range and a
+ * rebuild (steps 1-2) is due.  ws: any decode workspace (error word). */
+ABSP_API absp_status absp_append_centroids(const absp_layer_kv* kv, const absp_centroids* cent,
+                                           int32_t* exceeded, void* ws, size_t ws_bytes,
+                                           void* stream);
+
 /* Steps 3-4 (Fig. 1 "dot product estimation", "importance score",
  * "top-K selection"): for every (seq, kv_head), qbar = sum of the GQA
  * group's queries (q: device bf16 [S][Hq][128]), score[b] =
@@ -197,8 +213,12 @@ ABSP_API absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centro
                              const void* q, int32_t budget_tokens, void* out,
                              void* ws, size_t ws_bytes, void* stream);
 
-/* Flags of absp_decode_step_ex. */
+/* Flags of absp_decode_step_ex / absp_score_select_ex. */
 #define ABSP_STEP_EARLY_PREFETCH 1u
+#define ABSP_STEP_GROUP_MAX 2u
+/* ABSP_STEP_GROUP_MAX: the variant aggregation of a GQA group's queries: a
+ * block's score is max_j q_j . centroid over the group's query heads
+ * (fp32 per head) instead of qbar . centroid with qbar the group sum. */
 /* ABSP_STEP_EARLY_PREFETCH: the launch overlaps the tail of the preceding
  * kernel in `stream` (programmatic dependent launch) and, before waiting for
  * it, already reads the sequence lengths, page table, centroid codes and
@@ -209,12 +229,19 @@ ABSP_API absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centro
  * earlier steps, the query by the kernel just before.  Without the flag
  * nothing is read before the preceding kernel has completed. */
 
-/* absp_decode_step with flags (0 or ABSP_STEP_EARLY_PREFETCH); same
- * results as absp_decode_step. */
+/* absp_decode_step with flags (ABSP_STEP_EARLY_PREFETCH, ABSP_STEP_GROUP_MAX;
+ * other bits are rejected).  Without ABSP_STEP_GROUP_MAX, same results as
+ * absp_decode_step. */
 ABSP_API absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                          const void* q, int32_t budget_tokens, void* out,
                                          void* ws, size_t ws_bytes, uint32_t flags,
                                          void* stream);
+
+/* absp_score_select with flags (0 or ABSP_STEP_GROUP_MAX). */
+ABSP_API absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* cent,
+                                          const void* q, int32_t budget_tokens, int32_t* sel,
+                                          int32_t* sel_count, void* ws, size_t ws_bytes,
+                                          uint32_t flags, void* stream);
 
 /* absp_decode_step with HOST query and output buffers: copies q_host
  * (bf16 [S][Hq][128], pinned for true asynchrony) into the workspace, runs

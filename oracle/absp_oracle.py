@@ -147,6 +147,32 @@ def quantize_centroids(cent: np.ndarray) -> QuantizedCentroids:
     return QuantizedCentroids(codes, scale, zp)
 
 
+def append_tail_row(keys: np.ndarray, bs: int, scale: np.ndarray, zp: np.ndarray):
+    """Incremental update after appending tokens: the centroid of the block
+    that holds the last token, recomputed from that block's keys, and its
+    INT4 codes under the per-channel parameters of an earlier build.
+
+    Returns (block index, centroid fp64 [128], codes uint8 [128], number of
+    channels whose unclamped code fell outside 0..15, i.e. whose range the
+    earlier parameters no longer cover; channels with scale 0 carry no
+    information and are not counted).
+    """
+    L = keys.shape[0]
+    b = (L - 1) // bs
+    t0 = b * bs
+    acc = np.zeros(HEAD_DIM, dtype=np.float64)
+    for t in range(t0, L):
+        acc = acc + keys[t]
+    c = acc / (L - t0)
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    z = np.asarray(zp, dtype=np.int64).astype(np.float64)
+    live = s > 0
+    q = np.where(live, np.rint(c / np.where(live, s, 1.0)) + z, 0.0)
+    codes = np.clip(q, 0.0, float(CODE_LEVELS)).astype(np.uint8)
+    exceeded = int(np.count_nonzero(live & ((q < 0.0) | (q > CODE_LEVELS))))
+    return b, c, codes, exceeded
+
+
 def dequantize(qc: QuantizedCentroids) -> np.ndarray:
     """(code - zp) * scale, fp64."""
     return (qc.codes.astype(np.float64) - qc.zp.astype(np.float64)[None, :]) \
@@ -272,15 +298,29 @@ def head_keys_values(layer, s, h):
     return keys, vals
 
 
+def group_max_scores(cent_hat: np.ndarray, q_heads: np.ndarray, kv_head: int,
+                     group: int) -> np.ndarray:
+    """Variant aggregation: each block's score is the largest of the group's
+    per-head dot products q_j . centroid."""
+    qs = q_heads[kv_head * group:(kv_head + 1) * group]
+    return np.max(cent_hat @ qs.T, axis=1) if cent_hat.shape[0] else \
+        np.zeros(0, dtype=np.float64)
+
+
 def decode_head(q_heads: np.ndarray, kv_head: int, group: int, chat: np.ndarray,
                 keys: np.ndarray, values: np.ndarray, bs: int, seq_len: int,
-                budget: int, sel_override=None):
+                budget: int, sel_override=None, aggregate: str = "sum"):
     """Steps 3-5 for one (sequence, KV head) from its (dequantised) centroids.
 
+    aggregate="sum" scores with the group-summed query (the default
+    reading); "max" with the largest per-head score (the variant).
     Returns (scores, k, sel, outputs [group][128]).
     """
-    qbar = group_query(q_heads, kv_head, group)
-    sc = block_scores(chat, qbar)
+    if aggregate == "max":
+        sc = group_max_scores(chat, q_heads, kv_head, group)
+    else:
+        qbar = group_query(q_heads, kv_head, group)
+        sc = block_scores(chat, qbar)
     k = min(blocks_per_head(budget, bs), chat.shape[0])
     sel = select_blocks(sc, k)
     use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)
@@ -292,7 +332,8 @@ def decode_head(q_heads: np.ndarray, kv_head: int, group: int, chat: np.ndarray,
 
 
 def run_layer(layer, quantize=True, sel_override=None,
-              heads=None, with_attention: bool = True) -> LayerResult:
+              heads=None, with_attention: bool = True,
+              aggregate: str = "sum") -> LayerResult:
     """All five steps for every (sequence, KV head) of a host layer.
 
     `layer` carries q_bits [S][Hq][128], k_bits / v_bits
@@ -323,7 +364,8 @@ def run_layer(layer, quantize=True, sel_override=None,
                 chat = dequantize(qc) if quantize else cent
             ov = None if sel_override is None else sel_override[(s, h)]
             sc, k, sel, outs = decode_head(qf, h, G, chat, keys, vals, bs, L,
-                                           layer.budget, sel_override=ov)
+                                           layer.budget, sel_override=ov,
+                                           aggregate=aggregate)
             res.heads[(s, h)] = HeadResult(L, bs, cent, qc, sc, k, sel)
             if with_attention:
                 res.out[s, h * G:(h + 1) * G] = outs

@@ -159,6 +159,42 @@ def test_code_is_nearest_level_brute_force():
         assert q.codes[i, 0] == best
 
 
+def test_append_tail_row_equals_rebuild_row_within_range():
+    # appending tokens and re-quantising the tail block with the old
+    # parameters gives the full rebuild's row whenever the new centroid stays
+    # inside the old per-channel range
+    rng = np.random.default_rng(12)
+    keys = O.decode_bf16(_bf16_bits(rng.standard_normal((200, 128))))
+    bs = 16
+    old = O.quantize_centroids(O.build_centroids(keys[:180], bs))
+    b, c, codes, exc = O.append_tail_row(keys[:181], bs, old.scale, old.zp)
+    assert b == 11                                   # token 180 is in block 11
+    full = O.build_centroids(keys[:181], bs)
+    assert np.array_equal(c, full[11])
+    cd = old.codes.astype(np.float64)
+    s = old.scale.astype(np.float64)
+    want = np.clip(np.rint(full[11] / s) + old.zp, 0, 15)
+    assert np.array_equal(codes, want.astype(np.uint8))
+    # a single-token block closes the previous one: block 12 holds token 192
+    b2, c2, _, _ = O.append_tail_row(keys[:193], bs, old.scale, old.zp)
+    assert b2 == 12 and np.array_equal(c2, keys[192])
+    assert exc >= 0
+
+
+def test_append_tail_row_flags_out_of_range_channels():
+    keys = np.zeros((17, 128))
+    keys[:16, 0] = np.linspace(-1.0, 1.0, 16)        # block 0
+    keys[:16, 1] = 0.5
+    scale = np.full(128, np.float32(0.1))
+    zp = np.full(128, 5, dtype=np.int32)
+    keys[16, 0] = 100.0                              # far above code 15
+    keys[16, 1] = -0.2                               # code 3: inside
+    b, c, codes, exc = O.append_tail_row(keys, 16, scale, zp)
+    assert b == 1 and codes[0] == 15 and codes[1] == 3 and exc == 1
+    scale[0] = 0.0                                   # degenerate channel: not counted
+    assert O.append_tail_row(keys, 16, scale, zp)[3] == 0
+
+
 def test_pack_nibble_order_round_trip():
     codes = np.arange(128, dtype=np.uint8).reshape(1, 128) % 16
     p = O.pack_codes(codes)
@@ -201,6 +237,23 @@ def test_group_query_and_score_equal_sum_of_per_head_dots():
         want = [sum(float(np.dot(q[j], keys[t])) for j in range(h * G, h * G + G))
                 for t in range(20)]
         np.testing.assert_allclose(sc, want, rtol=1e-12, atol=1e-12)
+
+
+def test_group_max_is_max_of_per_head_dots_and_sum_bound():
+    rng = np.random.default_rng(14)
+    G, Hkv = 4, 2
+    q = rng.standard_normal((G * Hkv, 128))
+    c = rng.standard_normal((25, 128))
+    for h in range(Hkv):
+        got = O.group_max_scores(c, q, h, G)
+        for b in range(25):
+            dots = [float(np.dot(q[j], c[b])) for j in range(h * G, h * G + G)]
+            assert got[b] == pytest.approx(max(dots), rel=1e-12, abs=1e-12)
+        # the summed-query score never exceeds G times the max
+        assert np.all(O.block_scores(c, O.group_query(q, h, G)) <= G * got + 1e-9)
+    # with a group of one the two aggregations coincide
+    np.testing.assert_allclose(O.group_max_scores(c, q, 3, 1),
+                               O.block_scores(c, O.group_query(q, 3, 1)), rtol=1e-12)
 
 
 def test_score_is_linear_in_query():

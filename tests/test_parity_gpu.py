@@ -32,7 +32,8 @@ def _bits(t):
     return t.contiguous().view(torch.int16)
 
 
-def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None, fmt=0):
+def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None, fmt=0,
+             flags=0):
     abi, pipeline = lib
     d = data if data is not None else synth.make_layer(w, layer, "cuda")
     if modify is not None:
@@ -40,17 +41,17 @@ def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None, fm
     dl = pipeline.DeviceLayer(d, budget, fmt=fmt)
     bf16 = fmt == abi.ABSP_CENTROIDS_BF16
     dl.build_centroids()
-    dl.score_select()
+    dl.score_select(flags=flags)
     dl.sparse_decode()
     dl.check()
     out_split = dl.out.clone()
     dl.out.zero_()
-    dl.decode_step()
+    dl.decode_step(flags=flags)
     dl.check()
     torch.cuda.synchronize()
     assert torch.equal(_bits(dl.out), _bits(out_split)), "fused step != select + decode"
     dl.out.zero_()
-    dl.decode_step(flags=abi.ABSP_STEP_EARLY_PREFETCH)
+    dl.decode_step(flags=flags | abi.ABSP_STEP_EARLY_PREFETCH)
     dl.check()
     torch.cuda.synchronize()
     assert torch.equal(_bits(dl.out), _bits(out_split)), "early-prefetch step differs"
@@ -62,7 +63,8 @@ def run_case(lib, w, layer=0, seqs=None, modify=None, budget=None, data=None, fm
     sel = dl.sel.cpu().numpy()
     cnt = dl.sel_count.cpu().numpy()
     override = {(i, h): sel[s, h, :cnt[s, h]] for i, s in enumerate(seqs) for h in range(Hkv)}
-    res = O.run_layer(hl, quantize="bf16" if bf16 else True, sel_override=override)
+    res = O.run_layer(hl, quantize="bf16" if bf16 else True, sel_override=override,
+                      aggregate="max" if flags & abi.ABSP_STEP_GROUP_MAX else "sum")
     rep = PR.Report()
     for i, s in enumerate(seqs):
         for h in range(Hkv):
@@ -183,6 +185,25 @@ def test_bf16_centroids_ragged_gqa16(lib):
 def test_bf16_centroids_llama31_8b_32k(lib):
     abi, _ = lib
     run_case(lib, synth.WORKLOADS["llama31_8b_32k"], fmt=abi.ABSP_CENTROIDS_BF16)
+
+
+# ------------------------------------------- group-max aggregation variant --
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_group_max_tiny(lib, fmt):
+    abi, _ = lib
+    run_case(lib, synth.WORKLOADS["tiny_8k"], fmt=fmt, flags=abi.ABSP_STEP_GROUP_MAX)
+
+
+def test_group_max_ragged_gqa16(lib):
+    abi, _ = lib
+    w = synth.custom("gmax_ragged", 3, 32, 2, [3000, 77, 1025], [32, 16], 384, seed=61)
+    run_case(lib, w, flags=abi.ABSP_STEP_GROUP_MAX)
+
+
+def test_group_max_llama31_8b_32k(lib):
+    abi, _ = lib
+    run_case(lib, synth.WORKLOADS["llama31_8b_32k"], flags=abi.ABSP_STEP_GROUP_MAX)
 
 
 def test_host_buffers_match_device_step(lib):
