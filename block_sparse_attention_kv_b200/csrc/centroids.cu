@@ -273,20 +273,36 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
         const int b = (len - 1) / bs;
         const int t0 = b * bs;
         const int32_t* pt = kv.page_table + static_cast<int64_t>(s) * kv.max_pages;
+        // page ids of the block first (at most 4), then each page's rows
+        // with 16 loads in flight, summed in token order
+        int phys[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) phys[i] = t0 + i * kPage < len ? pt[t0 / kPage + i] : 0;
         double a[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int t = t0; t < len; ++t) {
-            const int phys = pt[t / kPage];
-            if (phys < 0 || phys >= kv.num_phys_pages) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int tp = t0 + i * kPage;
+            if (tp >= len) break;
+            const int nt = min(kPage, len - tp);
+            if (phys[i] < 0 || phys[i] >= kv.num_phys_pages) {
                 if (lane == 0) set_error(err, ABSP_ERR_DEVICE_FAULT, s);
                 continue;
             }
-            const uint2 v = ld_nc_u2(kv.k_pages +
-                                     ((static_cast<int64_t>(phys) * kv.Hkv + h) * kPage + t % kPage) * kD +
-                                     lane * 4);
-            a[0] += static_cast<double>(bf16lo(v.x));
-            a[1] += static_cast<double>(bf16hi(v.x));
-            a[2] += static_cast<double>(bf16lo(v.y));
-            a[3] += static_cast<double>(bf16hi(v.y));
+            const __nv_bfloat16* src =
+                kv.k_pages + ((static_cast<int64_t>(phys[i]) * kv.Hkv + h) * kPage) * kD + lane * 4;
+            uint2 v[kPage];
+#pragma unroll
+            for (int t = 0; t < kPage; ++t)
+                if (t < nt) v[t] = ld_nc_u2(src + t * kD);
+#pragma unroll
+            for (int t = 0; t < kPage; ++t) {
+                if (t < nt) {
+                    a[0] += static_cast<double>(bf16lo(v[t].x));
+                    a[1] += static_cast<double>(bf16hi(v[t].x));
+                    a[2] += static_cast<double>(bf16lo(v[t].y));
+                    a[3] += static_cast<double>(bf16hi(v[t].y));
+                }
+            }
         }
         const double cnt = static_cast<double>(len - t0);
         const int64_t row = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h] + b;
