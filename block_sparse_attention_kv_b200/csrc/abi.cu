@@ -132,6 +132,16 @@ bool use_pdl() {
     return v == 1;
 }
 
+// Device address of a pinned, device-mapped host buffer, else nullptr.
+void* mapped_host(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 absp_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
     if (ws == nullptr || !aligned(ws, kAlign)) return ABSP_ERR_INVALID_ARG;
     if (ws_bytes < need) return ABSP_ERR_INVALID_ARG;
@@ -364,6 +374,13 @@ absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids*
     if (st != ABSP_OK) return st;
     if ((st = check_ws(ws, ws_bytes, decode_ws_bytes(d))) != ABSP_OK) return st;
     if (q_host == nullptr || out_host == nullptr) return ABSP_ERR_INVALID_ARG;
+    // pinned host buffers mapped into the device address space: the kernel
+    // reads the query and writes the output across the host link itself
+    void* qm = mapped_host(q_host);
+    void* om = mapped_host(out_host);
+    if (qm != nullptr && om != nullptr && aligned(qm, 4) && aligned(om, 4))
+        return run_decode(kModeFull, kv, cent, qm, budget_tokens, nullptr, nullptr, om, ws,
+                          ws_bytes, stream);
     const size_t act = static_cast<size_t>(d.S) * d.Hq * ABSP_HEAD_DIM * 2;
     uint8_t* qd = static_cast<uint8_t*>(ws) + kWsHeader;
     uint8_t* od = qd + round_up(act, kAlign);

@@ -243,9 +243,12 @@ ABSP_API absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_ce
                                           int32_t* sel_count, void* ws, size_t ws_bytes,
                                           uint32_t flags, void* stream);
 
-/* absp_decode_step with HOST query and output buffers: copies q_host
- * (bf16 [S][Hq][128], pinned for true asynchrony) into the workspace, runs
- * the step and copies the result back to out_host, all on `stream`.  The
+/* absp_decode_step with HOST query and output buffers (bf16 [S][Hq][128]).
+ * When both are pinned and mapped into the device address space (pinned
+ * allocations are, under unified addressing), the kernel reads q_host and
+ * writes out_host directly across the host link; otherwise q_host is copied
+ * into the workspace, the step runs, and the result is copied back to
+ * out_host, all on `stream` (pin the buffers for true asynchrony).  The
  * caller synchronises `stream` before reading out_host. */
 ABSP_API absp_status absp_decode_step_host(const absp_layer_kv* kv,
                                   const absp_centroids* cent, const void* q_host,
