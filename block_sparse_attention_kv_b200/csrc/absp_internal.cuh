@@ -110,6 +110,11 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// Bulk prefetch of `bytes` (a multiple of 16; p 16-byte aligned) into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Wait for phase `parity` of an mbarrier, giving up after ~1 s.  On timeout
 // the error word records ABSP_ERR_TIMEOUT and the caller carries on (so that
 // every later cluster barrier is still reached); results are then garbage

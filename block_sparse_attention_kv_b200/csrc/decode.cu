@@ -38,6 +38,10 @@
 
 #include "absp_internal.cuh"
 
+#ifndef ABSP_PAGE_PREFETCH
+#define ABSP_PAGE_PREFETCH 2  // pages a warp prefetches into L2 ahead of its TMA copies
+#endif
+
 namespace absp {
 
 namespace {
@@ -45,10 +49,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kStageRows = 256;                      // code rows per bulk stage
-constexpr int kStages = 2;
+constexpr int kStages = 2;                           // ring stages in region A
+constexpr int kMaxStages = 4;                        // plus up to 2 in region B's free tail
 constexpr int kStageBytes = kStageRows * kRowBytes;  // 16 KiB
 constexpr int kPageSmem = 4 * 2048;                  // K lo/hi, V lo/hi halves
-constexpr int kMaxSlots = 2;                         // page buffers per warp
 constexpr int kBins = 1024;                          // value histogram
 constexpr int kMaxCand = 1024;                       // boundary-bin candidates
 constexpr int kMaxBitmapWords = (ABSP_MAX_BLOCKS_PER_HEAD + 31) / 32;
@@ -71,9 +75,10 @@ struct Params {
     uint32_t regA_off;            // byte offsets inside the aligned smem base
     uint32_t small_off;
     uint32_t scratch_off;         // select scratch inside region B
-    int32_t slots;                // page buffers per warp (1 or 2)
     int32_t group_max;            // score = max over the group's heads
     uint32_t wg_off;              // per-head weights inside region B
+    int32_t nstages;              // code ring stages (kStages .. kMaxStages)
+    uint32_t xstage_off;          // ring stages past kStages inside region B
 };
 
 // per-head score weights for the group-max variant: [G][8 lanes][20]
@@ -81,8 +86,8 @@ struct Params {
 constexpr int kWgStride = 160;
 
 struct Small {                    // fixed-size shared scratch
-    unsigned long long bar_code[kStages];
-    unsigned long long bar_page[kWarps][kMaxSlots];
+    unsigned long long bar_code[kMaxStages];
+    unsigned long long bar_page[kWarps];
     unsigned long long bar_merge;
     unsigned long long bar_score;
     float2 cmm[16];               // (min, max) of each cluster CTA's scores
@@ -90,6 +95,7 @@ struct Small {                    // fixed-size shared scratch
     float red[2][kWarps];
     float w[kD];                  // qbar[ch] * scale[ch]
     float zb[kD];                 // 2^23 + zp[ch]
+    float zf[kD];                 // zp[ch]
     uint32_t scan[kWarps];
 };
 
@@ -105,6 +111,57 @@ __device__ __forceinline__ int value_bin(float x, float mn, float inv) {
 
 __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
     return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// (a0, a1) += (w0, w1) * ((r0, r1) - 2^23), as packed f32x2 arithmetic; the
+// r are 2^23 + k for integers 0 <= k < 2^23, so the subtraction is exact.
+__device__ __forceinline__ void fma2_unbias(float& a0, float& a1, uint32_t r0, uint32_t r1,
+                                            float w0, float w1) {
+    asm("{\n\t.reg .b64 t, w, c;\n\t"
+        "mov.b64 t, {%2, %3};\n\t"
+        "mov.b64 w, {%4, %5};\n\t"
+        "mov.b64 c, {%0, %1};\n\t"
+        "sub.rn.f32x2 t, t, %6;\n\t"
+        "fma.rn.f32x2 c, w, t, c;\n\t"
+        "mov.b64 {%0, %1}, c;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(r0), "r"(r1), "f"(w0), "f"(w1), "l"(0x4B0000004B000000ull));
+}
+
+// Dot product of 16 INT4 codes (channel k in nibble k of x.x, then x.y) with
+// weights.  Nibble j (0..3) of each 16-bit half is masked in place and ORed
+// under the exponent of 2^23, which gives the float 2^23 + 16^j * code
+// exactly; w[k] carries the matching factor 16^-j (an exact power-of-two
+// scaling), so every product equals weight * code as if formed directly.
+// Two shifts per 16 channels instead of one per channel.
+__device__ __forceinline__ float int4_dot16(uint2 x, const float (&w)[16], float init) {
+    constexpr uint32_t M = 0x4B000000u;
+    const uint32_t h[4] = {x.x, x.x >> 16, x.y, x.y >> 16};
+    float a0 = init, a1 = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        fma2_unbias(a0, a1, (h[q] & 0xFu) | M, (h[q] & 0xF0u) | M, w[4 * q], w[4 * q + 1]);
+        fma2_unbias(a0, a1, (h[q] & 0xF00u) | M, (h[q] & 0xF000u) | M, w[4 * q + 2], w[4 * q + 3]);
+    }
+    return a0 + a1;
+}
+
+// Sums of four rows' partial dot products over the 8 lanes of a group
+// (lanes 8g .. 8g + 7), returned to every lane of the group.  A transpose
+// reduction: each butterfly step halves the rows a lane carries, so lane
+// 8g + j ends with the full sum of row j / 2 after three shuffles (instead of
+// three per row), then four shuffles gather the rows.
+__device__ __forceinline__ float4 group_sum4(const float (&a)[4], int lane) {
+    const bool hi = (lane & 4) != 0, mid = (lane & 2) != 0;
+    float k0 = hi ? a[2] : a[0], k1 = hi ? a[3] : a[1];
+    k0 += __shfl_xor_sync(0xffffffffu, hi ? a[0] : a[2], 4);
+    k1 += __shfl_xor_sync(0xffffffffu, hi ? a[1] : a[3], 4);
+    float k = mid ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, mid ? k0 : k1, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    const int base = lane & ~7;
+    return make_float4(__shfl_sync(0xffffffffu, k, base), __shfl_sync(0xffffffffu, k, base + 2),
+                       __shfl_sync(0xffffffffu, k, base + 4), __shfl_sync(0xffffffffu, k, base + 6));
 }
 
 // Block-wide exclusive prefix sum of one uint32 per thread (one barrier;
@@ -382,7 +439,6 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     const int pair = blockIdx.x / C;
     const int Hkv = p.kv.Hkv, G = p.kv.G;
     const int s = pair / Hkv, h = pair % Hkv;
-    const int NB = p.slots;
     const int bs = p.kv.bs[h];
     const int spb = bs / kPage;
     const int32_t* pt = p.kv.page_table + static_cast<int64_t>(s) * p.kv.max_pages;
@@ -393,9 +449,8 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     constexpr int kSRows = kStageBytes / kRow;         // rows per bulk stage
 
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
-        for (int w = 0; w < kWarps; ++w)
-            for (int i = 0; i < kMaxSlots; ++i) mbar_init(smem_u32(&sm.bar_page[w][i]), 1);
+        for (int i = 0; i < kMaxStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
+        for (int w = 0; w < kWarps; ++w) mbar_init(smem_u32(&sm.bar_page[w]), 1);
         mbar_init(smem_u32(&sm.bar_score), 1);
         if (C > 1) mbar_init(smem_u32(&sm.bar_merge), C - 1);
         fence_mbar_init();
@@ -418,17 +473,30 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     const int nchunks = (nrows + kSRows - 1) / kSRows;
     const uint8_t* cbase =
         p.codes + (static_cast<int64_t>(s) * p.kv.rows_per_seq + p.kv.row_base[h] + r0) * kRow;
+    // code ring: stages 0, 1 in region A, further ones in region B past the
+    // scores and select scratch (free until the attention phase)
+    const int NS = p.nstages;
+    auto stage_buf = [&](int st) -> uint8_t* {
+        return st < kStages ? regA + st * kStageBytes
+                            : regB + p.xstage_off + (st - kStages) * kStageBytes;
+    };
     if (tid == 0) {
         if (kSelect && (MODE != kModeSelect || rank == 0))
-            mbar_arrive_expect_tx(smem_u32(&sm.bar_score), 16 * ((n + 3) / 4) + 8 * C);
+            // every CTA's scores but this one's own (plain stores), and
+            // every CTA's (min, max)
+            mbar_arrive_expect_tx(smem_u32(&sm.bar_score),
+                                  16 * ((n + 3) / 4 - (nrows + 3) / 4) + 8 * C);
         if (kSelect) {
-            for (int c = 0; c < min(nchunks, kStages); ++c) {
+            for (int c = 0; c < min(nchunks, NS); ++c) {
                 const int rows = min(kSRows, nrows - c * kSRows);
                 const uint32_t bar = smem_u32(&sm.bar_code[c]);
                 mbar_arrive_expect_tx(bar, rows * kRow);
-                bulk_g2s(smem_u32(regA + c * kStageBytes), cbase + c * kStageBytes,
-                         rows * kRow, bar);
+                bulk_g2s(smem_u32(stage_buf(c)), cbase + c * kStageBytes, rows * kRow, bar);
             }
+            // the stages past the ring come from L2 when the ring refills
+            for (int c = NS; c < nchunks; ++c)
+                bulk_prefetch_l2(cbase + c * kStageBytes,
+                                 static_cast<uint32_t>(min(kSRows, nrows - c * kSRows) * kRow));
         }
     }
     // B0 arrive (release: the barrier set-up above is visible cluster-wide
@@ -468,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             for (int j = 0; j < G; ++j) qb += __bfloat162float(qh[j * kD]);
             sm.w[tid] = BF16C ? qb : qb * scl;
             sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
+            sm.zf[tid] = static_cast<float>(zpv);
             if (p.group_max) {
                 float* wg = reinterpret_cast<float*>(regB + p.wg_off);
                 const int slot = (tid >> 4) * 20 + (tid & 15);
@@ -480,10 +549,20 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         __syncthreads();
         const int sub = tid & 7, grp = tid >> 3;  // 32 groups of 8 lanes
         float wr[16], zr[16];
+        float kz = 0.0f;  // this lane's share of sum_ch w[ch] * zp[ch]
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             wr[k] = sm.w[sub * 16 + k];
             zr[k] = sm.zb[sub * 16 + k];
+        }
+        if (!BF16C && !p.group_max) {
+            // INT4 sum scores: sum_ch w (code - zp) = sum_ch w code - sum_ch w zp,
+            // with w pre-scaled for the in-place nibble extraction
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                kz = fmaf(wr[k], sm.zf[sub * 16 + k], kz);
+                wr[k] *= __uint_as_float(0x3F800000u - ((k & 3) << 25));  // 16^-(k mod 4)
+            }
         }
         float* scores = reinterpret_cast<float*>(regB);
         const uint32_t scores_u32 = smem_u32(scores);
@@ -494,129 +573,150 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             uint32_t* hist = reinterpret_cast<uint32_t*>(regB + p.scratch_off);
             for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
         }
-        for (int c = 0; c < nchunks; ++c) {
-            const int stage = c % kStages;
-            mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / kStages) & 1, p.err, 1);
-            const int rows = min(kSRows, nrows - c * kSRows);
-            const uint8_t* sbuf = regA + stage * kStageBytes;
-            // each 8-lane group scores 4 consecutive rows
-            for (int rb = 0; rb < rows; rb += 4 * (kThreads / 8)) {
-                const int r4 = rb + 4 * grp;
-                float q4[4];
+        // The chunk loop over the code ring; score4(sbuf, r4, rows) gives one
+        // 8-lane group's scores of rows r4 .. r4 + 3 of a stage (values for
+        // rows past `rows` are discarded here).
+        auto chunk_loop = [&](auto&& score4) {
+            for (int c = 0; c < nchunks; ++c) {
+                const int stage = c % NS;
+                mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / NS) & 1, p.err, 1);
+                const int rows = min(kSRows, nrows - c * kSRows);
+                const uint8_t* sbuf = stage_buf(stage);
+                for (int rb = 0; rb < rows; rb += 4 * (kThreads / 8)) {
+                    const int r4 = rb + 4 * grp;
+                    const float4 q = score4(sbuf, r4, rows);
+                    float q4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (r4 + u < rows) {
+                            lmin = fminf(lmin, q4[u]);
+                            lmax = fmaxf(lmax, q4[u]);
+                        } else {
+                            q4[u] = 0.0f;
+                        }
+                    }
+                    if (r4 < rows) {
+                        // to this CTA by a plain store, to the others by
+                        // st.async (which counts the bytes on their mbarrier)
+                        const uint32_t off = 4u * static_cast<uint32_t>(r0 + c * kSRows + r4);
+                        for (uint32_t dst = sub; dst < (MODE == kModeSelect ? 1u : C); dst += 8) {
+                            if (dst == rank)
+                                *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(scores) + off) =
+                                    make_float4(q4[0], q4[1], q4[2], q4[3]);
+                            else
+                                st_async_v4(dsmem_addr(scores_u32 + off, dst), q4[0], q4[1], q4[2],
+                                            q4[3], dsmem_addr(bar_score, dst));
+                        }
+                    }
+                }
+                __syncthreads();
+                if (tid == 0 && c + NS < nchunks) {
+                    const int cn = c + NS;
+                    const int rows_n = min(kSRows, nrows - cn * kSRows);
+                    const uint32_t bar = smem_u32(&sm.bar_code[stage]);
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(bar, rows_n * kRow);
+                    bulk_g2s(smem_u32(sbuf), cbase + cn * kStageBytes, rows_n * kRow, bar);
+                }
+            }
+        };
+        // The variant is uniform over the launch: each gets its own loop, so
+        // the four rows of a group are independent chains (no branch between
+        // them) and their sums take one transpose-reduction.
+        if (!p.group_max) {
+            if constexpr (BF16C) {
+                chunk_loop([&](const uint8_t* sbuf, int r4, int rows) {
+                    float a[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        // 16 bf16 centroid channels per lane: score += qbar * c
+                        uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
+                        if (r4 + u < rows) {
+                            const uint4* src =
+                                reinterpret_cast<const uint4*>(sbuf + (r4 + u) * kRow + sub * 32);
+                            y0 = src[0];
+                            y1 = src[1];
+                        }
+                        const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            acc = fmaf(wr[2 * k], bf16lo(yy[k]), acc);
+                            acc = fmaf(wr[2 * k + 1], bf16hi(yy[k]), acc);
+                        }
+                        a[u] = acc;
+                    }
+                    return group_sum4(a, lane);
+                });
+            } else {
+                chunk_loop([&](const uint8_t* sbuf, int r4, int rows) {
+                    float a[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        uint2 x = make_uint2(0u, 0u);
+                        if (r4 + u < rows)
+                            x = *reinterpret_cast<const uint2*>(sbuf + (r4 + u) * kRow + sub * 8);
+                        a[u] = int4_dot16(x, wr, -kz);
+                    }
+                    return group_sum4(a, lane);
+                });
+            }
+        } else {
+            chunk_loop([&](const uint8_t* sbuf, int r4, int rows) {
+                float sc[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int r = r4 + u;
-                    float acc = 0.0f;
-                    if (!p.group_max) {
-                        if constexpr (BF16C) {
-                            // 16 bf16 centroid channels per lane: score += qbar * c
-                            uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
-                            if (r < rows) {
-                                const uint4* src = reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
-                                y0 = src[0];
-                                y1 = src[1];
-                            }
-                            const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                acc = fmaf(wr[2 * k], bf16lo(yy[k]), acc);
-                                acc = fmaf(wr[2 * k + 1], bf16hi(yy[k]), acc);
-                            }
-                        } else {
-                            uint2 x = make_uint2(0u, 0u);
-                            if (r < rows) x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                const float f =
-                                    __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
-                                acc = fmaf(wr[k], f, acc);
-                            }
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                const float f =
-                                    __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
-                                acc = fmaf(wr[8 + k], f, acc);
-                            }
+                    float acc;
+                    // variant: the largest of the group's per-head scores
+                    float f[16];
+                    if constexpr (BF16C) {
+                        uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
+                        if (r < rows) {
+                            const uint4* src =
+                                reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
+                            y0 = src[0];
+                            y1 = src[1];
                         }
-                        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                        const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            f[2 * k] = bf16lo(yy[k]);
+                            f[2 * k + 1] = bf16hi(yy[k]);
+                        }
                     } else {
-                        // variant: the largest of the group's per-head scores
-                        float f[16];
-                        if constexpr (BF16C) {
-                            uint4 y0 = make_uint4(0u, 0u, 0u, 0u), y1 = y0;
-                            if (r < rows) {
-                                const uint4* src =
-                                    reinterpret_cast<const uint4*>(sbuf + r * kRow + sub * 32);
-                                y0 = src[0];
-                                y1 = src[1];
-                            }
-                            const uint32_t yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                        uint2 x = make_uint2(0u, 0u);
+                        if (r < rows)
+                            x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                f[2 * k] = bf16lo(yy[k]);
-                                f[2 * k + 1] = bf16hi(yy[k]);
-                            }
-                        } else {
-                            uint2 x = make_uint2(0u, 0u);
-                            if (r < rows)
-                                x = *reinterpret_cast<const uint2*>(sbuf + r * kRow + sub * 8);
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                f[k] = __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
-                                f[8 + k] =
-                                    __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
-                            }
-                        }
-                        const float* wg = reinterpret_cast<const float*>(regB + p.wg_off) + sub * 20;
-                        acc = -INFINITY;
-                        for (int jh = 0; jh < G; ++jh) {
-                            const float4* w4 = reinterpret_cast<const float4*>(wg + jh * kWgStride);
-                            float a = 0.0f;
-#pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4) {
-                                const float4 wv = w4[k4];
-                                a = fmaf(wv.x, f[4 * k4], a);
-                                a = fmaf(wv.y, f[4 * k4 + 1], a);
-                                a = fmaf(wv.z, f[4 * k4 + 2], a);
-                                a = fmaf(wv.w, f[4 * k4 + 3], a);
-                            }
-                            a += __shfl_xor_sync(0xffffffffu, a, 1);
-                            a += __shfl_xor_sync(0xffffffffu, a, 2);
-                            a += __shfl_xor_sync(0xffffffffu, a, 4);
-                            acc = fmaxf(acc, a);
+                        for (int k = 0; k < 8; ++k) {
+                            f[k] = __uint_as_float(0x4B000000u | ((x.x >> (4 * k)) & 0xFu)) - zr[k];
+                            f[8 + k] =
+                                __uint_as_float(0x4B000000u | ((x.y >> (4 * k)) & 0xFu)) - zr[8 + k];
                         }
                     }
-                    q4[u] = r < rows ? acc : 0.0f;
-                    if (r < rows) {
-                        lmin = fminf(lmin, acc);
-                        lmax = fmaxf(lmax, acc);
+                    const float* wg = reinterpret_cast<const float*>(regB + p.wg_off) + sub * 20;
+                    acc = -INFINITY;
+                    for (int jh = 0; jh < G; ++jh) {
+                        const float4* w4 = reinterpret_cast<const float4*>(wg + jh * kWgStride);
+                        float a = 0.0f;
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const float4 wv = w4[k4];
+                            a = fmaf(wv.x, f[4 * k4], a);
+                            a = fmaf(wv.y, f[4 * k4 + 1], a);
+                            a = fmaf(wv.z, f[4 * k4 + 2], a);
+                            a = fmaf(wv.w, f[4 * k4 + 3], a);
+                        }
+                        a += __shfl_xor_sync(0xffffffffu, a, 1);
+                        a += __shfl_xor_sync(0xffffffffu, a, 2);
+                        a += __shfl_xor_sync(0xffffffffu, a, 4);
+                        acc = fmaxf(acc, a);
                     }
+                    sc[u] = acc;
                 }
-                if (r4 < rows) {
-                    const uint32_t off = 4u * static_cast<uint32_t>(r0 + c * kSRows + r4);
-                    if (MODE == kModeSelect) {
-                        if (sub == 0)
-                            st_async_v4(dsmem_addr(scores_u32 + off, 0), q4[0], q4[1], q4[2],
-                                        q4[3], dsmem_addr(bar_score, 0));
-                    } else {
-                        for (uint32_t dst = sub; dst < C; dst += 8)
-                            st_async_v4(dsmem_addr(scores_u32 + off, dst), q4[0], q4[1], q4[2],
-                                        q4[3], dsmem_addr(bar_score, dst));
-                    }
-                }
-            }
-            __syncthreads();
-            if (tid == 0 && c + kStages < nchunks) {
-                const int cn = c + kStages;
-                const int rows_n = min(kSRows, nrows - cn * kSRows);
-                const uint32_t bar = smem_u32(&sm.bar_code[stage]);
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(bar, rows_n * kRow);
-                bulk_g2s(smem_u32(regA + stage * kStageBytes), cbase + cn * kStageBytes,
-                         rows_n * kRow, bar);
-            }
+                return make_float4(sc[0], sc[1], sc[2], sc[3]);
+            });
         }
         // this CTA's score range, sent along with the scores
 #pragma unroll
@@ -716,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         float m0 = -FLT_MAX, m8 = -FLT_MAX, l0 = 0.0f, l8 = 0.0f;
         bool any0 = false;  // this warp has seen at least one valid token
         const float qks = p.qk_scale_log2;
-        uint8_t* wbuf = regB + warp * NB * kPageSmem;  // this warp's page slots
+        uint8_t* wbuf = regB + warp * kPageSmem;  // this warp's page buffer
 
         // page i of this warp: selection entry, bounds checks, tensor copies
         auto issue = [&](int i) -> int {
@@ -738,13 +838,12 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                         valid = 0;
                     }
                 }
-                const int slot = i % NB;
-                const uint32_t bar = smem_u32(&sm.bar_page[warp][slot]);
+                const uint32_t bar = smem_u32(&sm.bar_page[warp]);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, valid > 0 ? kPageSmem : 0);
                 if (valid > 0) {
                     const int y = (phys * Hkv + h) * kPage;
-                    const uint32_t dst = smem_u32(wbuf + slot * kPageSmem);
+                    const uint32_t dst = smem_u32(wbuf);
                     tma_load_2d(dst, &tmk, 0, y, bar);
                     tma_load_2d(dst + 2048, &tmk, 64, y, bar);
                     tma_load_2d(dst + 4096, &tmv, 0, y, bar);
@@ -754,16 +853,30 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             return __shfl_sync(0xffffffffu, valid, 0);
         };
 
+        // page i of this warp: its K and V slices into L2, ahead of the copy
+        auto prefetch = [&](int i) {
+            if (lane != 0 || i >= cnt_w) return;
+            const int j = pb + warp + kWarps * i;
+            const int b = sel_s[j / spb - sel_lo];
+            if (b < 0) return;
+            const int lp = b * spb + (j % spb);
+            if (lp * kPage >= len) return;
+            const int phys = pt[lp];
+            if (phys < 0 || phys >= p.kv.num_phys_pages) return;
+            const int64_t off = (static_cast<int64_t>(phys) * Hkv + h) * (kPage * kD);
+            bulk_prefetch_l2(p.kv.k_pages + off, kPage * kD * 2);
+            bulk_prefetch_l2(p.kv.v_pages + off, kPage * kD * 2);
+        };
+
         __syncthreads();  // every thread is done with the scores in region B
-        int vq0 = 0, vq1 = 0;
-        if (cnt_w > 0) vq0 = issue(0);
-        if (NB > 1 && cnt_w > 1) vq1 = issue(1);
+        int vnext = cnt_w > 0 ? issue(0) : 0;
+#pragma unroll 1
+        for (int i = 1; i <= ABSP_PAGE_PREFETCH; ++i) prefetch(i);
         for (int i = 0; i < cnt_w; ++i) {
-            const int slot = i % NB;
-            const int valid = slot == 0 ? vq0 : vq1;
-            mbar_wait_bounded(smem_u32(&sm.bar_page[warp][slot]), (i / NB) & 1, p.err, 2);
+            const int valid = vnext;
+            mbar_wait_bounded(smem_u32(&sm.bar_page[warp]), i & 1, p.err, 2);
             if (valid > 0) {
-                uint8_t* pg = wbuf + slot * kPageSmem;
+                uint8_t* pg = wbuf;
                 const uint32_t kb = smem_u32(pg), vb = kb + 4096;
                 if (valid < kPage) {
                     // zero the V rows past the sequence end (they may hold
@@ -857,12 +970,10 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                     }
                 }
             }
-            fence_proxy_async_smem();  // this lane's reads/writes of the slot
-            __syncwarp();              // before the slot's next tensor copy
-            if (i + NB < cnt_w) {
-                const int v = issue(i + NB);
-                if (slot == 0) vq0 = v; else vq1 = v;
-            }
+            fence_proxy_async_smem();  // this lane's reads/writes of the buffer
+            __syncwarp();              // before its next tensor copy
+            if (i + 1 < cnt_w) vnext = issue(i + 1);
+            if (ABSP_PAGE_PREFETCH > 0) prefetch(i + 1 + ABSP_PAGE_PREFETCH);
         }
         l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
         l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -874,7 +985,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         }
 
         // ------------------------------------------- E: merge partials --
-        __syncthreads();                                   // page slots are dead
+        __syncthreads();                                   // page buffers are dead
         float* Ow = reinterpret_cast<float*>(regB);        // [warps][G][128]
         float* mw = Ow + kWarps * G * kD;                  // [warps][G]
         float* lw = mw + kWarps * G;
@@ -1024,10 +1135,15 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
 
 }  // namespace
 
-// Cluster size: enough CTAs to cover the SMs about twice, at most 16.
+#ifndef ABSP_DECODE_CTAS_PER_SM
+#define ABSP_DECODE_CTAS_PER_SM 2   // CTA count the cluster size aims for, per SM
+#endif
+
+// Cluster size: enough CTAs to cover the SMs about ABSP_DECODE_CTAS_PER_SM
+// times, at most 16.
 static int pick_cluster(int pairs, int num_sms) {
     int C = 1;
-    while (C < 16 && pairs * C * 2 <= 2 * num_sms) C *= 2;
+    while (C < 16 && pairs * C * 2 <= ABSP_DECODE_CTAS_PER_SM * num_sms) C *= 2;
     return C;
 }
 
@@ -1068,7 +1184,6 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
         // region B: scores + select scratch, or this CTA's page slots, or the
         // warp merge; region A: code ring, or (CTA 0) the cluster merge
         size_t regB = 0, regA = 0, scratch = 0;
-        int slots = 1;
         if (do_select) {
             // score slots for every row, rounded up to whole groups of 4
             scratch = (static_cast<size_t>(a.nmax + 3) / 4) * 16;
@@ -1078,17 +1193,27 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
             regA = std::max(regA, static_cast<size_t>(kStages) * kStageBytes);
         }
         if (do_attend) {
-            const int pages_max = a.budget / kPage;         // pages selected per head
-            const int per_cta = (pages_max + C - 1) / C;
-            slots = per_cta > kWarps ? kMaxSlots : 1;
-            regB = std::max(regB, static_cast<size_t>(kWarps) * slots * kPageSmem);
+            // one page buffer per warp: a second one (double buffering)
+            // halves the resident CTAs per SM and was slower on every
+            // workload measured
+            regB = std::max(regB, static_cast<size_t>(kWarps) * kPageSmem);
             regB = std::max(regB, static_cast<size_t>(kWarps) * G * (kD + 2) * 4);
             if (C > 1) regA = std::max(regA, static_cast<size_t>(C) * G * (kD + 2) * 4);
         }
         regB = (regB + 1023) & ~static_cast<size_t>(1023);
         regA = (regA + 127) & ~static_cast<size_t>(127);
+        // extra code-ring stages in what region B leaves free while scoring
+        prm.nstages = kStages;
+        prm.xstage_off = 0;
+        if (do_select) {
+            const size_t used = scratch + kSelectScratch +
+                                (a.group_max ? static_cast<size_t>(G) * kWgStride * 4 : 0);
+            const size_t off = (used + 127) & ~static_cast<size_t>(127);
+            const size_t extra = regB > off ? (regB - off) / kStageBytes : 0;
+            prm.nstages = kStages + static_cast<int>(std::min<size_t>(kMaxStages - kStages, extra));
+            prm.xstage_off = static_cast<uint32_t>(off);
+        }
         prm.scratch_off = static_cast<uint32_t>(scratch);
-        prm.slots = slots;
         prm.regA_off = static_cast<uint32_t>(regB);
         prm.small_off = static_cast<uint32_t>(regB + regA);
         const size_t smem = 1024 + regB + regA + sizeof(Small) + static_cast<size_t>(a.kmax) * 4;
