@@ -113,35 +113,34 @@ __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
     return *reinterpret_cast<const uint32_t*>(p);
 }
 
-// (a0, a1) += (w0, w1) * ((r0, r1) - 2^23), as packed f32x2 arithmetic; the
-// r are 2^23 + k for integers 0 <= k < 2^23, so the subtraction is exact.
-__device__ __forceinline__ void fma2_unbias(float& a0, float& a1, uint32_t r0, uint32_t r1,
-                                            float w0, float w1) {
+// (a0, a1) += (w0, w1) * (r0, r1) as one packed f32x2 FMA, r given as bits.
+__device__ __forceinline__ void fma2_bits(float& a0, float& a1, uint32_t r0, uint32_t r1,
+                                          float w0, float w1) {
     asm("{\n\t.reg .b64 t, w, c;\n\t"
         "mov.b64 t, {%2, %3};\n\t"
         "mov.b64 w, {%4, %5};\n\t"
         "mov.b64 c, {%0, %1};\n\t"
-        "sub.rn.f32x2 t, t, %6;\n\t"
         "fma.rn.f32x2 c, w, t, c;\n\t"
         "mov.b64 {%0, %1}, c;\n\t}"
         : "+f"(a0), "+f"(a1)
-        : "r"(r0), "r"(r1), "f"(w0), "f"(w1), "l"(0x4B0000004B000000ull));
+        : "r"(r0), "r"(r1), "f"(w0), "f"(w1));
 }
 
 // Dot product of 16 INT4 codes (channel k in nibble k of x.x, then x.y) with
-// weights.  Nibble j (0..3) of each 16-bit half is masked in place and ORed
-// under the exponent of 2^23, which gives the float 2^23 + 16^j * code
-// exactly; w[k] carries the matching factor 16^-j (an exact power-of-two
-// scaling), so every product equals weight * code as if formed directly.
-// Two shifts per 16 channels instead of one per channel.
+// weights, plus `init`.  Nibble j (0..3) of each 16-bit half is masked in
+// place; read as a float, the bits n * 16^j are the subnormal n * 16^j *
+// 2^-149, exactly.  w[k] carries the matching 2^(149 - 4j) (times the lane's
+// own power-of-two scale), so every product is weight * code times that
+// scale, formed exactly as if the code were a float: one AND per channel and
+// half a packed FMA, no conversion or unbias step.  Subnormal operands are
+// exact and full speed in fma.rn (no .ftz).
 __device__ __forceinline__ float int4_dot16(uint2 x, const float (&w)[16], float init) {
-    constexpr uint32_t M = 0x4B000000u;
     const uint32_t h[4] = {x.x, x.x >> 16, x.y, x.y >> 16};
     float a0 = init, a1 = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        fma2_unbias(a0, a1, (h[q] & 0xFu) | M, (h[q] & 0xF0u) | M, w[4 * q], w[4 * q + 1]);
-        fma2_unbias(a0, a1, (h[q] & 0xF00u) | M, (h[q] & 0xF000u) | M, w[4 * q + 2], w[4 * q + 3]);
+        fma2_bits(a0, a1, h[q] & 0xFu, h[q] & 0xF0u, w[4 * q], w[4 * q + 1]);
+        fma2_bits(a0, a1, h[q] & 0xF00u, h[q] & 0xF000u, w[4 * q + 2], w[4 * q + 3]);
     }
     return a0 + a1;
 }
@@ -549,20 +548,31 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         __syncthreads();
         const int sub = tid & 7, grp = tid >> 3;  // 32 groups of 8 lanes
         float wr[16], zr[16];
-        float kz = 0.0f;  // this lane's share of sum_ch w[ch] * zp[ch]
+        float kz = 0.0f;  // this lane's share of sum_ch w[ch] * zp[ch], scaled
+        float xs = 1.0f;  // 2^X: undoes the lane's scale on its partial sum
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             wr[k] = sm.w[sub * 16 + k];
             zr[k] = sm.zb[sub * 16 + k];
         }
         if (!BF16C && !p.group_max) {
-            // INT4 sum scores: sum_ch w (code - zp) = sum_ch w code - sum_ch w zp,
-            // with w pre-scaled for the in-place nibble extraction
+            // INT4 sum scores: sum_ch w (code - zp) = sum_ch w code - sum_ch w zp.
+            // The lane works at scale 2^-X, X from its largest |w| (2^e <=
+            // max|w| < 2^(e+1)): the pre-scaled weights w 2^(149 - 4j - X)
+            // stay below 2^126 and products of the larger weights are normal.
+            float mw = 0.0f;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 kz = fmaf(wr[k], sm.zf[sub * 16 + k], kz);
-                wr[k] *= __uint_as_float(0x3F800000u - ((k & 3) << 25));  // 16^-(k mod 4)
+                mw = fmaxf(mw, fabsf(wr[k]));
             }
+            const int e = static_cast<int>((__float_as_uint(mw) >> 23) & 0xFFu) - 127;
+            const int X = min(126, max(22, 24 + e));
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                wr[k] *= __uint_as_float(static_cast<uint32_t>(276 - X - 4 * (k & 3)) << 23);
+            kz *= __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
+            xs = __uint_as_float(static_cast<uint32_t>(127 + X) << 23);
         }
         float* scores = reinterpret_cast<float*>(regB);
         const uint32_t scores_u32 = smem_u32(scores);
@@ -656,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                         uint2 x = make_uint2(0u, 0u);
                         if (r4 + u < rows)
                             x = *reinterpret_cast<const uint2*>(sbuf + (r4 + u) * kRow + sub * 8);
-                        a[u] = int4_dot16(x, wr, -kz);
+                        a[u] = int4_dot16(x, wr, -kz) * xs;
                     }
                     return group_sum4(a, lane);
                 });
