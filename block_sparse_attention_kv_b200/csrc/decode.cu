@@ -86,6 +86,7 @@ struct Params {
 constexpr int kWgStride = 160;
 
 struct Small {                    // fixed-size shared scratch
+    __nv_bfloat16 qs[ABSP_MAX_GROUP * kD];  // the group's queries (full mode)
     unsigned long long bar_code[kMaxStages];
     unsigned long long bar_page[kWarps];
     unsigned long long bar_merge;
@@ -97,6 +98,9 @@ struct Small {                    // fixed-size shared scratch
     float zb[kD];                 // 2^23 + zp[ch]
     float zf[kD];                 // zp[ch]
     uint32_t scan[kWarps];
+    float fw[ABSP_MAX_GROUP * kWarps];  // warp merge: exp2(m_w - M) per (row, warp)
+    float rowM[ABSP_MAX_GROUP];          //   and the row's M and L
+    float rowL[ABSP_MAX_GROUP];
 };
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -143,6 +147,34 @@ __device__ __forceinline__ float int4_dot16(uint2 x, const float (&w)[16], float
         fma2_bits(a0, a1, h[q] & 0xF00u, h[q] & 0xF000u, w[4 * q + 2], w[4 * q + 3]);
     }
     return a0 + a1;
+}
+
+// Softmax merge weights of n partials (m_i, l_i) per row, n a power of two
+// <= 32, for `rows` rows: partial i of row r is at [i * rows + r].  One
+// thread per (row, partial) pair, the pairs of a row on n consecutive lanes;
+// every thread of the block calls this.  Writes f[r * n + i] = exp2(m_i - M)
+// (normalised by 1 / L when `normalise`) and, when given, M and L per row,
+// with M = max_i m_i and L = sum_i l_i exp2(m_i - M); a row with no valid
+// token (M = -inf) gets zero weights.
+__device__ __forceinline__ void merge_factors(const float* m, const float* l, int rows, int n,
+                                              float* f, float* rowM, float* rowL, bool normalise) {
+    const int tid = threadIdx.x;
+    const int pairs = rows * n;
+    if (tid >= ((pairs + 31) & ~31)) return;  // whole warps only (full-mask shuffles)
+    const bool act = tid < pairs;
+    const int row = act ? tid / n : 0, i = act ? tid % n : 0;
+    const float mi = act ? m[i * rows + row] : -INFINITY;
+    float M = mi;
+    for (int o = 1; o < n; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float e = M != -INFINITY ? exp2f(mi - M) : 0.0f;
+    float L = act ? l[i * rows + row] * e : 0.0f;
+    for (int o = 1; o < n; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (!act) return;
+    f[row * n + i] = normalise ? (L > 0.0f ? e * (1.0f / L) : 0.0f) : e;
+    if (rowM != nullptr && i == 0) {
+        rowM[row] = M;
+        rowL[row] = L;
+    }
 }
 
 // Sums of four rows' partial dot products over the 8 lanes of a group
@@ -531,8 +563,14 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         K = min(n, max(1, p.budget / bs));
         if (tid < kD) {
             const __nv_bfloat16* qh = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD + tid;
+            // the group's queries are read once (they may live in host
+            // memory) and kept for the attention phase
             float qb = 0.0f;
-            for (int j = 0; j < G; ++j) qb += __bfloat162float(qh[j * kD]);
+            for (int j = 0; j < G; ++j) {
+                const __nv_bfloat16 qv = qh[j * kD];
+                sm.qs[j * kD + tid] = qv;
+                qb += __bfloat162float(qv);
+            }
             sm.w[tid] = BF16C ? qb : qb * scl;
             sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
             sm.zf[tid] = static_cast<float>(zpv);
@@ -540,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                 float* wg = reinterpret_cast<float*>(regB + p.wg_off);
                 const int slot = (tid >> 4) * 20 + (tid & 15);
                 for (int j = 0; j < G; ++j) {
-                    const float qj = __bfloat162float(qh[j * kD]);
+                    const float qj = __bfloat162float(sm.qs[j * kD + tid]);
                     wg[j * kWgStride + slot] = BF16C ? qj : qj * scl;
                 }
             }
@@ -756,9 +794,12 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
 
         // --------------------------------------------------- C: select --
         float smin = INFINITY, smax = -INFINITY;
-        for (uint32_t r = 0; r < C; ++r) {
-            smin = fminf(smin, sm.cmm[r].x);
-            smax = fmaxf(smax, sm.cmm[r].y);
+#pragma unroll
+        for (uint32_t r = 0; r < 16; ++r) {  // C <= 16; independent loads
+            if (r < C) {
+                smin = fminf(smin, sm.cmm[r].x);
+                smax = fmaxf(smax, sm.cmm[r].y);
+            }
         }
         if (MODE == kModeSelect) {
             sel_lo = 0;
@@ -767,8 +808,8 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             // this CTA attends list entries [sel_lo, sel_hi): the blocks of
             // its share [pb, pe) of the K * bs/16 selected pages
             const int P = K * spb;
-            const int pb = static_cast<int>((static_cast<int64_t>(P) * rank) / C);
-            const int pe = static_cast<int>((static_cast<int64_t>(P) * (rank + 1)) / C);
+            const int pb = static_cast<int>(static_cast<uint32_t>(P) * rank / C);  // P*C < 2^21
+            const int pe = static_cast<int>(static_cast<uint32_t>(P) * (rank + 1) / C);
             sel_lo = pb / spb;
             sel_hi = pe > pb ? (pe - 1) / spb + 1 : sel_lo;
         }
@@ -802,11 +843,13 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     if constexpr ((MODE & kModeAttend) != 0) {
         // --------------------------------------------------- D: attend --
         const int P = K * spb;
-        const int pb = static_cast<int>((static_cast<int64_t>(P) * rank) / C);
-        const int pe = static_cast<int>((static_cast<int64_t>(P) * (rank + 1)) / C);
+        const int pb = static_cast<int>(static_cast<uint32_t>(P) * rank / C);  // P*C < 2^21
+        const int pe = static_cast<int>(static_cast<uint32_t>(P) * (rank + 1) / C);
         const int cnt_w = pe - pb > warp ? (pe - pb - warp + kWarps - 1) / kWarps : 0;
         const int g = lane >> 2, t4 = lane & 3;
-        const __nv_bfloat16* qg = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
+        // queries: the copy made while scoring, else (attend only) global
+        const __nv_bfloat16* qg =
+            kSelect ? sm.qs : p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
         uint32_t qa0[8], qa2[8], qa1[8], qa3[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -1024,6 +1067,10 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             }
         }
         __syncthreads();
+        // per (row, warp) weight exp2(m_w - M) and the row's M and L: one
+        // thread per pair, reduced over the warp's 8-lane segment
+        merge_factors(mw, lw, G, kWarps, sm.fw, sm.rowM, sm.rowL, false);
+        __syncthreads();
         if constexpr ((MODE & kModeSelect) == 0) cluster_wait();  // B0
         float* partO = reinterpret_cast<float*>(regA);    // [C][G][128]
         float* partM = partO + C * G * kD;                 // [C][G]
@@ -1031,16 +1078,14 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         __nv_bfloat16* outp = p.out + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
         for (int idx = tid; idx < G * kD; idx += kThreads) {
             const int row = idx >> 7, d = idx & (kD - 1);
-            float M = -INFINITY;
-            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mw[w * G + row]);
-            float L = 0.0f, Oacc = 0.0f;
-            if (M != -INFINITY) {
-                for (int w = 0; w < kWarps; ++w) {
-                    const float f = exp2f(mw[w * G + row] - M);
-                    L += lw[w * G + row] * f;
-                    Oacc += Ow[(w * G + row) * kD + d] * f;
-                }
+            const float M = sm.rowM[row], L = sm.rowL[row];
+            float oa = 0.0f, ob = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; w += 2) {
+                oa = fmaf(Ow[(w * G + row) * kD + d], sm.fw[row * kWarps + w], oa);
+                ob = fmaf(Ow[((w + 1) * G + row) * kD + d], sm.fw[row * kWarps + w + 1], ob);
             }
+            const float Oacc = oa + ob;
             if (C == 1) {
                 outp[row * kD + d] = __float2bfloat16_rn(L > 0.0f ? Oacc / L : 0.0f);
             } else if (rank == 0) {
@@ -1066,24 +1111,24 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                 return;
             }
             mbar_wait_bounded<true>(smem_u32(&sm.bar_merge), 0, p.err, 3);
-            // per (row, partial) weight exp2(m_r - M) / L, computed once
+            // per (row, partial) weight exp2(m_r - M) / L: one thread per
+            // pair, reduced over the C-lane segment
             float* fac = Ow;                   // [G][C]; the warp partials are consumed
-            if (tid < G) {
-                float M = -INFINITY;
-                for (uint32_t r = 0; r < C; ++r) M = fmaxf(M, partM[r * G + tid]);
-                float L = 0.0f;
-                if (M != -INFINITY)
-                    for (uint32_t r = 0; r < C; ++r) L += partL[r * G + tid] * exp2f(partM[r * G + tid] - M);
-                const float invL = L > 0.0f ? 1.0f / L : 0.0f;
-                for (uint32_t r = 0; r < C; ++r)
-                    fac[tid * C + r] = M != -INFINITY ? exp2f(partM[r * G + tid] - M) * invL : 0.0f;
-            }
+            merge_factors(partM, partL, G, static_cast<int>(C), fac, nullptr, nullptr, true);
             __syncthreads();
             for (int idx = tid; idx < G * kD; idx += kThreads) {
                 const int row = idx >> 7, d = idx & (kD - 1);
-                float Oacc = 0.0f;
-                for (uint32_t r = 0; r < C; ++r) Oacc += partO[(r * G + row) * kD + d] * fac[row * C + r];
-                outp[row * kD + d] = __float2bfloat16_rn(Oacc);
+                const float* po = partO + row * kD + d;
+                const float* fr = fac + row * C;
+                float o4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                uint32_t r = 0;
+                for (; r + 4 <= C; r += 4) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        o4[i] = fmaf(po[(r + i) * G * kD], fr[r + i], o4[i]);
+                }
+                for (; r < C; ++r) o4[0] = fmaf(po[r * G * kD], fr[r], o4[0]);
+                outp[row * kD + d] = __float2bfloat16_rn((o4[0] + o4[1]) + (o4[2] + o4[3]));
             }
         }
     }
