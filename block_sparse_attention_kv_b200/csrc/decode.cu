@@ -75,7 +75,6 @@ struct Params {
     uint32_t regA_off;            // byte offsets inside the aligned smem base
     uint32_t small_off;
     uint32_t scratch_off;         // select scratch inside region B
-    int32_t group_max;            // score = max over the group's heads
     uint32_t wg_off;              // per-head weights inside region B
     int32_t nstages;              // code ring stages (kStages .. kMaxStages)
     uint32_t xstage_off;          // ring stages past kStages inside region B
@@ -230,7 +229,7 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v) {
 
 // Threshold of the top-k by 4 passes of 8-bit radix select over the
 // order-preserving keys (keys > T are in, plus `rem` keys equal to T).
-__device__ __forceinline__ void radix_threshold(const float* sc, int n, int k, uint32_t* hist, Small& sm,
+__device__ __noinline__ void radix_threshold(const float* sc, int n, int k, uint32_t* hist, Small& sm,
                                 uint32_t* T_out, int* rem_out) {
     const int tid = threadIdx.x;
     uint32_t prefix = 0, mask = 0;
@@ -267,7 +266,7 @@ __device__ __forceinline__ void radix_threshold(const float* sc, int n, int k, u
 // Ordered compaction of the top-k by a threshold: keys > T are in, and of
 // the keys == T the `rem` lowest indices.  Each warp compacts a contiguous
 // index range 32 scores at a time with ballots.
-__device__ __forceinline__ void compact_by_threshold(const float* sc, int n, uint32_t T, int rem,
+__device__ __noinline__ void compact_by_threshold(const float* sc, int n, uint32_t T, int rem,
                                                      int32_t* out, int lo, int hi, Small& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per_w = (n + kWarps - 1) / kWarps;
@@ -307,24 +306,26 @@ __device__ __forceinline__ void compact_by_threshold(const float* sc, int n, uin
 // bitmap[0..nwords), by one warp: out[pos - lo] = bit index.
 __device__ __forceinline__ void warp_extract_bitmap(const uint32_t* bitmap, int nwords,
                                                     int32_t* out, int lo, int hi) {
+    // run once per CTA by one warp: compact loops rather than unrolled ones
+    // keep this cold code small
     const int lane = threadIdx.x & 31;
     const int wpl = (nwords + 31) / 32;
     const int j0 = min(nwords, lane * wpl), j1 = min(nwords, j0 + wpl);
-    uint32_t words[16];
     uint32_t cnt = 0;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        words[u] = j0 + u < j1 ? bitmap[j0 + u] : 0u;
-        cnt += __popc(words[u]);
-    }
+#pragma unroll 1
+    for (int j = j0; j < j1; ++j) cnt += __popc(bitmap[j]);
     int pos = static_cast<int>(warp_excl_scan(cnt));
     if (pos + static_cast<int>(cnt) <= lo || pos >= hi) return;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        uint32_t bits = words[u];
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            if (pos >= lo && pos < hi) out[pos - lo] = (j0 + u) * 32 + b;
+#pragma unroll 1
+    for (int j = j0; j < j1 && pos < hi; ++j) {
+        uint32_t bits = bitmap[j];
+        const int c = __popc(bits);
+        if (pos + c <= lo) {  // the whole word lies before the wanted entries
+            pos += c;
+            continue;
+        }
+        while (bits && pos < hi) {
+            if (pos >= lo) out[pos - lo] = j * 32 + (__ffs(bits) - 1);
             ++pos;
             bits &= bits - 1u;
         }
@@ -451,7 +452,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 #define ABSP_DECODE_MIN_BLOCKS 2
 #endif
 
-template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C>
+template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM>
 __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             sm.w[tid] = BF16C ? qb : qb * scl;
             sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
             sm.zf[tid] = static_cast<float>(zpv);
-            if (p.group_max) {
+            if constexpr (GM) {
                 float* wg = reinterpret_cast<float*>(regB + p.wg_off);
                 const int slot = (tid >> 4) * 20 + (tid & 15);
                 for (int j = 0; j < G; ++j) {
@@ -593,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             wr[k] = sm.w[sub * 16 + k];
             zr[k] = sm.zb[sub * 16 + k];
         }
-        if (!BF16C && !p.group_max) {
+        if constexpr (!BF16C && !GM) {
             // INT4 sum scores: sum_ch w (code - zp) = sum_ch w code - sum_ch w zp.
             // The lane works at scale 2^-X, X from its largest |w| (2^e <=
             // max|w| < 2^(e+1)): the pre-scaled weights w 2^(149 - 4j - X)
@@ -671,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         // The variant is uniform over the launch: each gets its own loop, so
         // the four rows of a group are independent chains (no branch between
         // them) and their sums take one transpose-reduction.
-        if (!p.group_max) {
+        if constexpr (!GM) {
             if constexpr (BF16C) {
                 chunk_loop([&](const uint8_t* sbuf, int r4, int rows) {
                     float a[4];
@@ -1134,11 +1135,11 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     }
 }
 
-template <int MODE, bool BIG, bool EARLY, bool BF16C = false>
+template <int MODE, bool BIG, bool EARLY, bool BF16C, bool GM>
 cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool pdl,
                         const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st,
                         bool* fits) {
-    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C>;
+    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C, GM>;
     static bool configured = false;   // attributes are per function, set once
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1202,6 +1203,19 @@ static int pick_cluster(int pairs, int num_sms) {
     return C;
 }
 
+// centroid format x score aggregation: each pair is its own kernel, so the
+// default one (INT4, sum) carries no code of the others
+template <int MODE, bool BIG, bool EARLY>
+cudaError_t launch_variant(bool bf, bool gm, const Params& prm, size_t smem, int C, int pairs,
+                           bool pdl, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                           cudaStream_t st, bool* fits) {
+    if (bf)
+        return gm ? launch_mode<MODE, BIG, EARLY, true, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, fits)
+                  : launch_mode<MODE, BIG, EARLY, true, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, fits);
+    return gm ? launch_mode<MODE, BIG, EARLY, false, true>(prm, smem, C, pairs, pdl, tmk, tmv, st, fits)
+              : launch_mode<MODE, BIG, EARLY, false, false>(prm, smem, C, pairs, pdl, tmk, tmv, st, fits);
+}
+
 cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
                           const CUtensorMap* tmv, bool pdl, bool early_prefetch, cudaStream_t st) {
     static int num_sms = 0;
@@ -1230,7 +1244,6 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     prm.budget = a.budget;
     prm.err = a.err;
     prm.qk_scale_log2 = kLog2e / sqrtf(static_cast<float>(kD));
-    prm.group_max = a.group_max;
     prm.wg_off = 0;
 
     int C = pick_cluster(pairs, num_sms);
@@ -1275,29 +1288,28 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
         if (smem > 227 * 1024) return cudaErrorInvalidValue;
         bool fits = false;
         const bool early = early_prefetch && mode == kModeFull;
-#define ABSP_LAUNCH(M, B, E, F) \
-    launch_mode<M, B, E, F>(prm, smem, C, pairs, pdl, tmk, tmv, st, &fits)
-        const bool bf = a.cfmt == ABSP_CENTROIDS_BF16;
+        const bool bf = a.cfmt == ABSP_CENTROIDS_BF16, gm = a.group_max != 0;
         if (mode == kModeAttend) {
-            e = big ? ABSP_LAUNCH(kModeAttend, true, false, false)
-                    : ABSP_LAUNCH(kModeAttend, false, false, false);
+            e = big ? launch_mode<kModeAttend, true, false, false, false>(
+                          prm, smem, C, pairs, pdl, tmk, tmv, st, &fits)
+                    : launch_mode<kModeAttend, false, false, false, false>(
+                          prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
         } else if (mode == kModeSelect) {
-            if (big) e = bf ? ABSP_LAUNCH(kModeSelect, true, false, true)
-                            : ABSP_LAUNCH(kModeSelect, true, false, false);
-            else e = bf ? ABSP_LAUNCH(kModeSelect, false, false, true)
-                        : ABSP_LAUNCH(kModeSelect, false, false, false);
+            e = big ? launch_variant<kModeSelect, true, false>(bf, gm, prm, smem, C, pairs, pdl,
+                                                               tmk, tmv, st, &fits)
+                    : launch_variant<kModeSelect, false, false>(bf, gm, prm, smem, C, pairs, pdl,
+                                                                tmk, tmv, st, &fits);
         } else if (big) {
-            if (early) e = bf ? ABSP_LAUNCH(kModeFull, true, true, true)
-                              : ABSP_LAUNCH(kModeFull, true, true, false);
-            else e = bf ? ABSP_LAUNCH(kModeFull, true, false, true)
-                        : ABSP_LAUNCH(kModeFull, true, false, false);
+            e = early ? launch_variant<kModeFull, true, true>(bf, gm, prm, smem, C, pairs, pdl,
+                                                              tmk, tmv, st, &fits)
+                      : launch_variant<kModeFull, true, false>(bf, gm, prm, smem, C, pairs, pdl,
+                                                               tmk, tmv, st, &fits);
         } else {
-            if (early) e = bf ? ABSP_LAUNCH(kModeFull, false, true, true)
-                              : ABSP_LAUNCH(kModeFull, false, true, false);
-            else e = bf ? ABSP_LAUNCH(kModeFull, false, false, true)
-                        : ABSP_LAUNCH(kModeFull, false, false, false);
+            e = early ? launch_variant<kModeFull, false, true>(bf, gm, prm, smem, C, pairs, pdl,
+                                                               tmk, tmv, st, &fits)
+                      : launch_variant<kModeFull, false, false>(bf, gm, prm, smem, C, pairs, pdl,
+                                                                tmk, tmv, st, &fits);
         }
-#undef ABSP_LAUNCH
         if (e != cudaSuccess || fits) return e;
         // this cluster shape cannot be resident: retry with a smaller one
     }
