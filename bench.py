@@ -18,13 +18,17 @@ writes.  `variants.plain` is the same measurement with absp_decode_step
 
 value   = layer-steps/s over all ranks (weak scaling: every rank decodes its
           own layer stack, no collective on the data path);
-e2e     = the same through absp_decode_step_host (query copied from pinned
-          host memory and output copied back inside every layer-step);
+e2e     = the same through absp_decode_step_host with pinned host buffers
+          (the kernel reads each layer's query from host memory and writes
+          its output there, inside every layer-step);
 roofline= algorithmic bytes of a layer-step (centroid codes + per-channel
           parameters + valid selected K/V rows + q and out) / average launch
           time, against the measured HBM copy bandwidth;
 rebuild = centroid build + INT4 quantisation of every layer (steps 1-2),
-          timed separately (it runs once per cache, not per token).
+          timed separately (it runs once per cache, not per token);
+calibration = per-head normalised recall at block sizes 16/32/64 on a set of
+          heads of varied concentration, and the block-size allocation it
+          gives at the centroid memory of a uniform block size 32.
 
 `--impl reference` times the CPU oracle on the same workload instead.
 """
@@ -302,6 +306,37 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------ block-size calibration --
+
+def calibration_summary(dev, synth):
+    """Per-head sensitivity on the 8-head calibration set and the block-size
+    allocation it gives at the centroid memory of a uniform block size 32."""
+    from block_sparse_attention_kv_b200 import calibrate as cal
+    w = synth.WORKLOADS["calib_8h_32k"]
+    d = synth.make_layer(w, 0, dev)
+    t0 = time.perf_counter()
+    c = cal.calibrate(d, lambda s, h: synth.planted_mask(d.plan, s, h))
+    budget = int(c.rows[:, 1].sum())
+    choice, _, used = cal.allocate(c.normalised, c.rows, budget)
+    ms = (time.perf_counter() - t0) * 1e3
+    rec = c.recall
+    H = rec.shape[0]
+    del d
+    return {
+        "workload": "calib_8h_32k: 8 KV heads (32 q), 32K ctx, budget 2048, 512 planted "
+                    "q-aligned tokens per head in spans of 4 .. 512 tokens",
+        "span_tokens": [int(x) for x in w.planted_lens],
+        "block_sizes": list(c.block_sizes),
+        "normalised_recall": [[round(float(v), 4) for v in row] for row in c.normalised],
+        "recall_uniform": {str(bs): float(rec[:, j].mean()) for j, bs in enumerate(c.block_sizes)},
+        "alloc_budget_rows": budget,
+        "alloc_rows": int(used),
+        "alloc_block_sizes": [int(c.block_sizes[j]) for j in choice],
+        "recall_alloc": float(np.mean([rec[h, choice[h]] for h in range(H)])),
+        "ms": ms,
+    }
+
+
 # ----------------------------------------------------------- GPU arm --
 
 def gpu_arm(args):
@@ -356,6 +391,7 @@ def gpu_arm(args):
     rb_bytes = sum(rebuild_bytes(x.data) for x in layers) / L
     del bws
     rb_large = None if args.no_variants else rebuild_large(dev, stream, abi, pipeline, synth)
+    calib = None if args.no_variants or rank != 0 else calibration_summary(dev, synth)
 
     # algorithmic bytes from each layer's own selection
     nbytes = []
@@ -550,6 +586,7 @@ def gpu_arm(args):
                                "note": "absp_decode_step, no reads before the previous "
                                        "launch completes"}},
         "append": append,
+        "calibration": calib,
         "clocks": clocks,
         "rebuild": {"ms_per_layer": rebuild_ms, "bytes_per_layer": rb_bytes,
                     "achieved_gbs": rb_bytes / (rebuild_ms * 1e-3) / 1e9,

@@ -62,6 +62,11 @@ class Workload:
     planted_blocks: int = 8
     planted_len: int = 64
     planted_gain: float = 2.0
+    # per-KV-head span lengths (tokens): when given, head h gets
+    # planted_tokens // planted_lens[h] spans of that length at arbitrary
+    # token offsets (heads of different concentration); else the spans above
+    planted_lens: Optional[tuple] = None
+    planted_tokens: int = 512
     spare_pages: int = 0
     seed: int = 0
 
@@ -91,6 +96,13 @@ WORKLOADS = {
     "rebuild_8x128k": Workload("rebuild_8x128k", layers=1, num_seqs=8,
                                num_q_heads=32, num_kv_heads=8, ctx=131072,
                                budget=2048, seed=1005),
+    # Block-size sensitivity: 8 KV heads whose 512 relevant tokens come in
+    # spans of 4 .. 512 tokens (concentrated to spread), 32K context.
+    "calib_8h_32k": Workload("calib_8h_32k", layers=1, num_seqs=1,
+                             num_q_heads=32, num_kv_heads=8, ctx=32768,
+                             budget=2048, block_sizes=(16,) * 8,
+                             planted_lens=(4, 8, 16, 32, 64, 128, 256, 512),
+                             planted_tokens=512, seed=1006),
 }
 
 
@@ -146,6 +158,21 @@ def draw_seq_lens(w: Workload) -> np.ndarray:
     return np.clip(np.floor(np.exp(u)), lo, hi).astype(np.int32)
 
 
+def planted_len(w: Workload, h: int) -> int:
+    """Length of KV head h's planted spans (tokens)."""
+    return int(w.planted_lens[h]) if w.planted_lens is not None else int(w.planted_len)
+
+
+def planted_mask(plan: "LayerPlan", s: int, h: int) -> np.ndarray:
+    """Token mask of the planted (q-aligned) keys of (sequence s, KV head h)."""
+    L = int(plan.seq_lens[s])
+    m = np.zeros(L, dtype=bool)
+    ln = planted_len(plan.workload, h)
+    for st in plan.planted[s][h]:
+        m[int(st):min(L, int(st) + ln)] = True
+    return m
+
+
 def plan_layer(w: Workload, layer: int = 0) -> LayerPlan:
     S, Hkv = w.num_seqs, w.num_kv_heads
     lens = draw_seq_lens(w)
@@ -157,12 +184,21 @@ def plan_layer(w: Workload, layer: int = 0) -> LayerPlan:
     planted = []
     for s in range(S):
         row = []
-        nspan = int(lens[s]) // w.planted_len
-        for _h in range(Hkv):
-            k = min(w.planted_blocks, nspan)
-            starts = np.sort(r.choice(nspan, size=k, replace=False)) * w.planted_len \
-                if k > 0 else np.zeros(0, np.int64)
-            row.append(starts.astype(np.int64))
+        for h in range(Hkv):
+            if w.planted_lens is None:
+                nspan = int(lens[s]) // w.planted_len
+                k = min(w.planted_blocks, nspan)
+                starts = np.sort(r.choice(nspan, size=k, replace=False)) * w.planted_len \
+                    if k > 0 else np.zeros(0, np.int64)
+            else:
+                # spans of length ln at any offset inside disjoint 2*ln slots
+                ln = int(w.planted_lens[h])
+                nslot = int(lens[s]) // (2 * ln)
+                k = min(max(1, w.planted_tokens // ln), nslot)
+                slots = np.sort(r.choice(nslot, size=k, replace=False)) if k > 0 \
+                    else np.zeros(0, np.int64)
+                starts = slots * (2 * ln) + r.integers(0, ln + 1, size=k)
+            row.append(np.asarray(starts, dtype=np.int64))
         planted.append(row)
     pages_per_seq = [(int(L) + PAGE_SIZE - 1) // PAGE_SIZE for L in lens]
     max_pages = max(1, max(pages_per_seq))
@@ -244,9 +280,10 @@ def make_layer(w: Workload, layer: int = 0, device="cpu",
             bias.scatter_(1, outl, w.outlier_bias)
             kk += bias
         for h in range(Hkv):
+            ln = planted_len(w, h)
             for st in plan.planted[s][h]:
                 st = int(st)
-                kk[st:st + w.planted_len, h, :] += w.planted_gain * u[s, h]
+                kk[st:st + ln, h, :] += w.planted_gain * u[s, h]
         vv = torch.randn((L, Hkv, D), generator=g, device=dev,
                          dtype=torch.float32)
         pad = npg * PAGE_SIZE - L
