@@ -39,7 +39,11 @@ CODE_ROW_BYTES = 64
 class AbspError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = int(status)
-        super().__init__(f"{what}: {absp_status_string(status)} (status {status})")
+        msg = f"{what}: {absp_status_string(status)} (status {status})"
+        if self.status == ABSP_ERR_CUDA:   # which CUDA call failed, and how
+            self.cuda_error = absp_last_cuda_error()
+            msg += f": CUDA error {self.cuda_error} ({absp_last_cuda_error_string()})"
+        super().__init__(msg)
 
 
 class absp_layer_kv(Structure):
@@ -107,6 +111,8 @@ def _load() -> ctypes.CDLL:
         "absp_check_device_error": (st, [c_void_p, c_size_t, c_void_p, P(c_int32)]),
         "absp_build_quantize_noalloc": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p,
                                              c_void_p]),
+        "absp_last_cuda_error": (c_int32, []),
+        "absp_last_cuda_error_string": (c_char_p, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -124,7 +130,8 @@ EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_sizes_fm
             "absp_score_select_ex",
             "absp_sparse_decode",
             "absp_decode_step", "absp_decode_step_ex", "absp_decode_step_host",
-            "absp_check_device_error", "absp_build_quantize_noalloc")
+            "absp_check_device_error", "absp_build_quantize_noalloc",
+            "absp_last_cuda_error", "absp_last_cuda_error_string")
 
 
 def lib() -> ctypes.CDLL:
@@ -224,6 +231,14 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 def absp_status_string(status: int) -> str:
     return _lib.absp_status_string(int(status)).decode()
+
+
+def absp_last_cuda_error() -> int:
+    return int(_lib.absp_last_cuda_error())
+
+
+def absp_last_cuda_error_string() -> str:
+    return _lib.absp_last_cuda_error_string().decode()
 
 
 def absp_centroid_sizes(kv: LayerKV):

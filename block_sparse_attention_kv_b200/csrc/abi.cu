@@ -70,6 +70,16 @@ absp_status absp::make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v) {
 }
 
 namespace {
+thread_local int t_last_cuda = 0;  // last CUDA error turned into ABSP_ERR_CUDA here
+}  // namespace
+
+absp_status absp::cuda_status(int e) {
+    if (e == 0) return ABSP_OK;
+    t_last_cuda = e;
+    return ABSP_ERR_CUDA;
+}
+
+namespace {
 
 absp_status check_budget(const KvDesc& d, int32_t budget, int32_t* kmax, int32_t* nmax) {
     if (budget < ABSP_PAGE_SIZE || budget > ABSP_MAX_BUDGET) return ABSP_ERR_INVALID_ARG;
@@ -83,7 +93,7 @@ absp_status check_budget(const KvDesc& d, int32_t budget, int32_t* kmax, int32_t
     return ABSP_OK;
 }
 
-absp_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ABSP_OK : ABSP_ERR_CUDA; }
+absp_status from_cuda(cudaError_t e) { return cuda_status(static_cast<int>(e)); }
 
 // ----------------------------------------------------------- tensor maps --
 
@@ -105,8 +115,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 16 token rows x 64 channels (128 bytes, 128-byte swizzle), so one
 // (page, head) slice is two boxes.
 absp_status page_tensor_map(const void* pages, const KvDesc& d, CUtensorMap* m) {
+    // the encoding is a driver call: on a thread that has not used CUDA yet
+    // no context is current, so let the runtime bind the current device's
+    // context first (once per thread)
+    static thread_local bool bound = false;
+    if (!bound) {
+        const cudaError_t e = cudaFree(nullptr);
+        if (e != cudaSuccess) return from_cuda(e);
+        bound = true;
+    }
     auto fn = encode_fn();
-    if (fn == nullptr) return ABSP_ERR_CUDA;
+    if (fn == nullptr) return cuda_status(cudaErrorNotSupported);
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(ABSP_HEAD_DIM),
                           static_cast<cuuint64_t>(d.num_phys_pages) * d.Hkv * ABSP_PAGE_SIZE};
     cuuint64_t strides[1] = {ABSP_HEAD_DIM * 2};
@@ -115,7 +134,7 @@ absp_status page_tensor_map(const void* pages, const KvDesc& d, CUtensorMap* m) 
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pages), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? ABSP_OK : ABSP_ERR_CUDA;
+    return cuda_status(static_cast<int>(r));  // a driver code (same numbering for the usual ones)
 }
 
 size_t decode_ws_bytes(const KvDesc& d) {
@@ -124,12 +143,11 @@ size_t decode_ws_bytes(const KvDesc& d) {
 }
 
 bool use_pdl() {
-    static int v = -1;
-    if (v < 0) {
+    static const bool v = [] {  // read once (thread-safe initialisation)
         const char* e = std::getenv("ABSP_PDL");
-        v = (e != nullptr && e[0] == '0') ? 0 : 1;
-    }
-    return v == 1;
+        return !(e != nullptr && e[0] == '0');
+    }();
+    return v;
 }
 
 // Device address of a pinned, device-mapped host buffer, else nullptr.
@@ -386,7 +404,7 @@ absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids*
     uint8_t* od = qd + round_up(act, kAlign);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync(qd, q_host, act, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return ABSP_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     st = run_decode(kModeFull, kv, cent, qd, budget_tokens, nullptr, nullptr, od, ws, ws_bytes,
                     stream);
     if (st != ABSP_OK) return st;
@@ -398,14 +416,21 @@ absp_status absp_check_device_error(void* ws, size_t ws_bytes, void* stream, int
     if (ws == nullptr || ws_bytes < static_cast<size_t>(kWsHeader)) return ABSP_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t word[2] = {0, 0};
-    if (cudaMemcpyAsync(word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return ABSP_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return ABSP_ERR_CUDA;
+    cudaError_t e = cudaMemcpyAsync(word, ws, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return from_cuda(e);
     if (detail) *detail = word[1];
     if (word[0] == 0) return ABSP_OK;
-    if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return ABSP_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return ABSP_ERR_CUDA;
+    e = cudaMemsetAsync(ws, 0, sizeof(word), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return from_cuda(e);
     return word[0] == ABSP_ERR_TIMEOUT ? ABSP_ERR_TIMEOUT : ABSP_ERR_DEVICE_FAULT;
+}
+
+int absp_last_cuda_error(void) { return t_last_cuda; }
+
+const char* absp_last_cuda_error_string(void) {
+    return t_last_cuda == 0 ? "no error" : cudaGetErrorString(static_cast<cudaError_t>(t_last_cuda));
 }
 
 }  // extern "C"

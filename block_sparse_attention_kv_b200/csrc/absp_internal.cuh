@@ -280,6 +280,9 @@ __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v &
 
 // Checks a layer description and fills the kernel descriptor (abi.cu).
 absp_status make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v);
+// ABSP_OK for cudaSuccess; otherwise records `e` as the calling thread's last
+// CUDA error (absp_last_cuda_error) and returns ABSP_ERR_CUDA.
+absp_status cuda_status(int e);
 // Checks the three centroid buffers (abi.cu).
 absp_status check_cent(const absp_centroids* c);
 

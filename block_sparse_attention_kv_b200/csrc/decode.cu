@@ -34,7 +34,9 @@
 // Modes: select only (writes sel / sel_count), attend only (reads them) and
 // full (A-E in one launch, the selection never leaves the chip).
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
+#include <mutex>
 
 #include "absp_internal.cuh"
 
@@ -1135,19 +1137,53 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
     }
 }
 
+constexpr int kCacheDevices = 16;  // devices with cached launch state
+
+// the last 8 (cluster size, shared bytes) shapes asked about on one device
+struct ShapeCache {
+    int c[8] = {};
+    size_t smem[8] = {};
+    int fit[8] = {};
+    int next = 0;
+    int find(int C, size_t bytes) const {
+        for (int i = 0; i < 8; ++i)
+            if (c[i] == C && smem[i] == bytes) return fit[i];
+        return -1;
+    }
+    void insert(int C, size_t bytes, int f) {
+        c[next] = C;
+        smem[next] = bytes;
+        fit[next] = f;
+        next = (next + 1) & 7;
+    }
+};
+
 template <int MODE, bool BIG, bool EARLY, bool BF16C, bool GM>
 cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool pdl,
                         const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st,
                         bool* fits) {
     auto kern = decode_kernel<MODE, BIG, EARLY, BF16C, GM>;
-    static bool configured = false;   // attributes are per function, set once
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             227 * 1024);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        configured = true;
+    // per device (function attributes belong to a device's context) and
+    // per shape: whether one cluster of C CTAs with `smem` bytes fits
+    static std::mutex mu;
+    static bool configured[kCacheDevices] = {};
+    static ShapeCache shapes[kCacheDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < kCacheDevices;
+    int fit = -1;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!cached || !configured[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     227 * 1024);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            if (cached) configured[dev] = true;
+        }
+        if (cached) fit = shapes[dev].find(C, smem);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pairs * C);
@@ -1163,25 +1199,18 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // can at least one cluster of this shape be resident?  (cached per shape)
-    static int cache_c[8] = {0}, cache_fit[8] = {0};
-    static size_t cache_smem[8] = {0};
-    static int next = 0;
-    int fit = -1;
-    for (int i = 0; i < 8; ++i)
-        if (cache_c[i] == C && cache_smem[i] == smem) fit = cache_fit[i];
     if (fit < 0) {
+        // can one cluster of this shape be resident?  A failed query is not
+        // an answer: it is not cached and the launch below reports the error
+        std::lock_guard<std::mutex> lock(mu);
         int nclusters = 0;
-        cudaError_t e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
-        if (e != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess) {
+            fit = nclusters > 0 ? 1 : 0;
+            if (cached) shapes[dev].insert(C, smem, fit);
+        } else {
             cudaGetLastError();
-            nclusters = 0;
+            fit = 1;
         }
-        fit = nclusters > 0 ? 1 : 0;
-        cache_c[next] = C;
-        cache_smem[next] = smem;
-        cache_fit[next] = fit;
-        next = (next + 1) & 7;
     }
     *fits = fit != 0;
     if (!fit) return cudaSuccess;
@@ -1218,12 +1247,16 @@ cudaError_t launch_variant(bool bf, bool gm, const Params& prm, size_t smem, int
 
 cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
                           const CUtensorMap* tmv, bool pdl, bool early_prefetch, cudaStream_t st) {
-    static int num_sms = 0;
-    if (num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (num_sms <= 0) num_sms = 148;
+    static std::atomic<int> sms_of[kCacheDevices];  // SM count per device, 0 = unknown
+    int dev = 0, num_sms = 0;
+    cudaGetDevice(&dev);
+    const bool cached = dev >= 0 && dev < kCacheDevices;
+    if (cached) num_sms = sms_of[dev].load(std::memory_order_relaxed);
+    if (num_sms <= 0) {
+        if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            num_sms <= 0)
+            num_sms = 148;
+        if (cached) sms_of[dev].store(num_sms, std::memory_order_relaxed);
     }
     const int pairs = a.kv.S * a.kv.Hkv;
     const int G = a.kv.G;

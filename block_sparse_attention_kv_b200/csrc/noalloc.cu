@@ -62,19 +62,21 @@ extern "C" absp_status absp_build_quantize_noalloc(const absp_layer_kv* kv,
     if (absp::build_ws_bytes(d) > static_cast<size_t>(ABSP_NOALLOC_BUILD_WS_BYTES))
         return ABSP_ERR_UNSUPPORTED;
     void* ws = nullptr;
-    if (noalloc_scratch(&ws) != cudaSuccess) return ABSP_ERR_CUDA;
+    cudaError_t e = noalloc_scratch(&ws);
+    if (e != cudaSuccess) return absp::cuda_status(e);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the error word and detail start at zero; launch_build resets the
     // min/max keys itself
-    if (cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s) != cudaSuccess) return ABSP_ERR_CUDA;
+    if ((e = cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s)) != cudaSuccess)
+        return absp::cuda_status(e);
     const absp::BuildWs w = absp::build_ws_layout(ws, d);
-    if (absp::launch_build(d, w, s) != cudaSuccess) return ABSP_ERR_CUDA;
-    if (absp::launch_quantize(d, w, out->codes, out->scale, out->zp, out->format, s) !=
+    if ((e = absp::launch_build(d, w, s)) != cudaSuccess) return absp::cuda_status(e);
+    if ((e = absp::launch_quantize(d, w, out->codes, out->scale, out->zp, out->format, s)) !=
         cudaSuccess)
-        return ABSP_ERR_CUDA;
+        return absp::cuda_status(e);
     if (device_status != nullptr &&
-        cudaMemcpyAsync(device_status, ws, 2 * sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
-            cudaSuccess)
-        return ABSP_ERR_CUDA;
+        (e = cudaMemcpyAsync(device_status, ws, 2 * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                             s)) != cudaSuccess)
+        return absp::cuda_status(e);
     return ABSP_OK;
 }

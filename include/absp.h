@@ -288,6 +288,16 @@ ABSP_API absp_status absp_build_quantize_noalloc(const absp_layer_kv* kv,
 ABSP_API absp_status absp_check_device_error(void* ws, size_t ws_bytes, void* stream,
                                     int32_t* detail);
 
+/* The CUDA error behind the most recent ABSP_ERR_CUDA that a call of this
+ * library returned on the calling thread (0 if none yet): a cudaError_t, or
+ * for a tensor-map encoding failure the driver's CUresult (the two agree on
+ * the common codes).  Host only, never launches, never fails. */
+ABSP_API int absp_last_cuda_error(void);
+
+/* cudaGetErrorString of absp_last_cuda_error(), "no error" when it is 0.
+ * The string is static; do not free it. */
+ABSP_API const char* absp_last_cuda_error_string(void);
+
 #ifdef __cplusplus
 }
 #endif

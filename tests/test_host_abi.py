@@ -26,8 +26,8 @@ def abi():
 
 def _declared_symbols():
     txt = open(os.path.join(ROOT, "include", "absp.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:ABSP_API\s+)?(?:absp_status|const char\*)\s+(absp_\w+)\(",
-                                 txt, re.M)))
+    return sorted(set(re.findall(
+        r"^\s*(?:ABSP_API\s+)?(?:absp_status|const char\*|int)\s+(absp_\w+)\(", txt, re.M)))
 
 
 def test_header_declares_the_boundary():
@@ -35,6 +35,17 @@ def test_header_declares_the_boundary():
     for want in ("absp_build_centroids", "absp_quantize_centroids", "absp_score_select",
                  "absp_sparse_decode", "absp_decode_step"):
         assert want in names
+
+
+def test_last_cuda_error_starts_clear(abi):
+    # per thread; a thread that has seen no CUDA failure reads 0 / "no error"
+    import threading
+    seen = []
+    t = threading.Thread(target=lambda: seen.append((abi.absp_last_cuda_error(),
+                                                     abi.absp_last_cuda_error_string())))
+    t.start()
+    t.join()
+    assert seen == [(0, "no error")]
 
 
 def test_library_exports_every_declared_symbol(abi):

@@ -263,6 +263,49 @@ def test_repeated_steps_are_deterministic(lib):
     assert torch.equal(_bits(a), _bits(dl.out))
 
 
+def test_concurrent_host_threads(lib):
+    # the library's launch path (per-device caches, attribute set-up) driven
+    # from several host threads at once, each with its own stream and layer;
+    # every thread's results equal a serial run bit for bit
+    import threading
+    abi, pipeline = lib
+    ws = [synth.custom(f"mt{i}", 1, 8 * (1 + i % 2), 2, [3000 + 700 * i], [16, 64], 512,
+                       seed=300 + i) for i in range(4)]
+    layers, want, streams = [], [], []
+    for w in ws:
+        d = synth.make_layer(w, 0, "cuda")
+        streams.append(torch.cuda.Stream())
+        dl = pipeline.DeviceLayer(d, stream=streams[-1].cuda_stream)
+        dl.build_centroids()
+        torch.cuda.synchronize()
+        layers.append(dl)
+    for dl in layers:
+        dl.decode_step(flags=abi.ABSP_STEP_EARLY_PREFETCH)
+        torch.cuda.synchronize()
+        want.append(dl.out.clone())
+    errors = []
+
+    def work(dl):
+        try:
+            for i in range(25):
+                dl.decode_step(flags=abi.ABSP_STEP_EARLY_PREFETCH if i % 2 else 0)
+                dl.score_select()
+                dl.sparse_decode()
+        except Exception as e:  # reported by the main thread
+            errors.append(e)
+
+    ts = [threading.Thread(target=work, args=(dl,)) for dl in layers]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    torch.cuda.synchronize()
+    assert not errors, errors
+    for dl, w in zip(layers, want):
+        dl.check()
+        assert torch.equal(_bits(dl.out), _bits(w))
+
+
 # ----------------------------------------------------- device-side faults --
 
 def _fault_layer(lib):
