@@ -237,8 +237,9 @@ def rebuild_large(dev, stream, abi, pipeline, synth):
 
 # ------------------------------------------------------- CPU oracle leg --
 
-def oracle_layer_sample(layer_index: int = 0):
-    """Host copy of one layer plus the oracle's prebuilt centroids."""
+def oracle_layer_sample(layer_index: int = 0, heads=None):
+    """Host copy of one layer plus the oracle's prebuilt centroids (of the
+    KV heads in `heads`, all when None)."""
     from block_sparse_attention_kv_b200 import synth
     from oracle import absp_oracle as O
     w = synth.WORKLOADS[WORKLOAD]
@@ -248,6 +249,8 @@ def oracle_layer_sample(layer_index: int = 0):
     for s in range(hl.q_bits.shape[0]):
         qf = O.decode_bf16(hl.q_bits[s])
         for h in range(len(hl.block_size)):
+            if heads is not None and h not in heads:
+                continue
             keys, vals = O.head_keys_values(hl, s, h)
             bs = int(hl.block_size[h])
             chat = O.dequantize(O.quantize_centroids(O.build_centroids(keys, bs)))
@@ -279,6 +282,36 @@ def time_oracle(prep, G, budget, steps: int = None, seconds: float = None):
     if lim is not None:
         lim.unregister() if hasattr(lim, "unregister") else None
     return done, el
+
+
+def _oracle_worker(task):
+    """One process of the all-cores oracle timing: (units done, seconds)."""
+    seconds, head, barrier = task
+    prep, G, budget = oracle_layer_sample(0, heads=[head])
+    barrier.wait()                      # every worker times the same window
+    return time_oracle(prep, G, budget, seconds=seconds)
+
+
+def time_oracle_all_cores(seconds: float, max_procs: int = 32):
+    """The oracle on one process per host core (at most max_procs), each on
+    one KV head of the workload's layer 0; spawn start, so it is safe after
+    the GPU was used.  Returns (layer-steps/s, processes, units, seconds)."""
+    import multiprocessing as mp
+    n = max(1, min(os.cpu_count() or 1, max_procs))
+    ctx = mp.get_context("spawn")
+    nh = synth_kv_heads()
+    with ctx.Manager() as mgr:
+        bar = mgr.Barrier(n)
+        with ctx.Pool(n) as pool:
+            res = pool.map(_oracle_worker, [(seconds, i % nh, bar) for i in range(n)])
+    units = sum(r[0] for r in res)
+    el = max(r[1] for r in res)
+    return (units / nh) / el, n, units, el
+
+
+def synth_kv_heads() -> int:
+    from block_sparse_attention_kv_b200 import synth
+    return synth.WORKLOADS[WORKLOAD].num_kv_heads
 
 
 def reference_arm(args):
@@ -544,6 +577,14 @@ def gpu_arm(args):
                "sample": f"{done} (sequence, KV head) decode units of one {WORKLOAD} layer "
                          f"({done / len(prep):.2f} layer-steps, steps 3-5 from prebuilt "
                          f"centroids), numpy fp64, 1 thread, {el:.1f} s"}
+        try:
+            v, n, units, el2 = time_oracle_all_cores(args.cpu_seconds)
+            cpu["all_cores"] = {
+                "value": v, "unit": UNIT, "cores": n, "kind": "oracle",
+                "sample": f"{units} decode units on {n} processes (one KV head of a "
+                          f"{WORKLOAD} layer each, 1 thread each), {el2:.1f} s window"}
+        except Exception as e:  # the single-thread figure above stands
+            cpu["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
 
     peak, peak_kind = hbm_peak()
     launch_ms = ms / (args.steps * L)
