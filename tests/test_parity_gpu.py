@@ -125,6 +125,15 @@ def test_gqa_groups(lib, hq, hkv):
     run_case(lib, w)
 
 
+def test_many_pairs_one_cta_each(lib):
+    # 80 (sequence, KV head) pairs: the launch gives each pair one CTA (no
+    # score exchange, no cluster merge); ragged lengths leave partial chunks
+    # and partial lane groups
+    lens = [1 + (977 * i) % 4100 for i in range(40)]
+    w = synth.custom("many_pairs", 40, 8, 2, lens, [16, 64], 512, seed=41)
+    run_case(lib, w)
+
+
 @pytest.mark.parametrize("bs", [16, 64])
 def test_uniform_block_size(lib, bs):
     w = synth.custom(f"uniform{bs}", 2, 16, 4, [5000, 3333], [bs] * 4, 1024, seed=20 + bs)
