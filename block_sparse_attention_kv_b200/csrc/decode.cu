@@ -6,12 +6,15 @@
 // One thread-block cluster of C CTAs (C in 1..16) handles one
 // (sequence, KV head).  Phases of decode_kernel:
 //   A  score:   CTA r streams its contiguous 1/C share of the head's code
-//               rows into shared memory with 1-D bulk copies, scores every
-//               row (8 lanes per 64-byte row, 16 codes per lane, fp32) and
-//               sends each group of 4 scores to every CTA of the cluster
-//               with asynchronous 16-byte distributed-shared-memory stores
-//               that count down the receiver's mbarrier.  Meanwhile the
-//               sequence's page-table row is prefetched into L2.
+//               rows into shared memory with 1-D bulk copies through a ring
+//               of 16 KB stages, scores every row (8 lanes per 64-byte row,
+//               16 codes per lane, 4 rows per lane group at once, codes fed
+//               to packed f32x2 FMAs as exact subnormals, fp32 sums) and
+//               sends each group of 4 scores to the other CTAs of the
+//               cluster with asynchronous 16-byte distributed-shared-memory
+//               stores that count down the receiver's mbarrier (its own
+//               scores with plain stores).  Meanwhile the sequence's
+//               page-table row is prefetched into L2.
 //   B  each CTA waits on its own mbarrier until all n_h scores arrived.
 //   C  select:  every CTA runs the same deterministic top-K (largest scores,
 //               ties to the lower block index): a 1024-bin histogram over the
@@ -27,12 +30,16 @@
 //               tensor copies (128-byte swizzle, no multicast) on its own
 //               mbarrier, then computes S^T = Q K^T and O += P V on mma.sync
 //               bf16 tiles with the GQA group as the 16-row M dimension and an
-//               online softmax in fp32.
+//               online softmax in fp32; each warp also bulk-prefetches its
+//               next two pages into L2.
 //   E  merge:   warps merge in shared memory; CTAs write their (m, l, O)
 //               partials into CTA 0 through distributed shared memory and
 //               arrive on CTA 0's mbarrier; CTA 0 merges and writes bf16.
 // Modes: select only (writes sel / sel_count), attend only (reads them) and
-// full (A-E in one launch, the selection never leaves the chip).
+// full (A-E in one launch, the selection never leaves the chip).  Centroid
+// format (INT4 / BF16) and score aggregation (sum / group max) are template
+// parameters, so the default kernel carries no code of the other variants
+// (its phases run once per launch and their code is fetched every time).
 #include <algorithm>
 #include <atomic>
 #include <cfloat>
