@@ -397,6 +397,24 @@ def test_qwen3_8b_128k_layer(lib, layer):
     run_case(lib, synth.WORKLOADS["qwen3_8b_128k_36l"], layer=layer)
 
 
+def test_max_blocks_per_head(lib):
+    # 262144 tokens at block size 16: head 0 holds ABSP_MAX_BLOCKS_PER_HEAD
+    # (16384) code rows, the largest score buffer and selection bitmap
+    abi, _ = lib
+    w = synth.custom("max_blocks", 1, 8, 2, [262144], [16, 64], 4096, seed=51)
+    rep, dl, res = run_case(lib, w)
+    assert res.heads[(0, 0)].centroids.shape[0] == 16384
+
+
+def test_max_budget(lib):
+    # the largest token budget (65536) over a 131072-token context: half of
+    # every head's blocks are selected, 32 pages per warp, the longest list
+    w = synth.custom("max_budget", 1, 8, 2, [131072], [16, 64], 65536, seed=52)
+    rep, dl, res = run_case(lib, w)
+    cnt = dl.sel_count.cpu().numpy()
+    assert cnt[0].tolist() == [4096, 1024]
+
+
 def test_batch32_32k_sampled(lib):
     run_case(lib, synth.WORKLOADS["batch32_32k_8l"], layer=3, seqs=[0, 17, 31])
 
