@@ -857,9 +857,16 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
         const int pe = static_cast<int>(static_cast<uint32_t>(P) * (rank + 1) / C);
         const int cnt_w = pe - pb > warp ? (pe - pb - warp + kWarps - 1) / kWarps : 0;
         const int g = lane >> 2, t4 = lane & 3;
-        // queries: the copy made while scoring, else (attend only) global
-        const __nv_bfloat16* qg =
-            kSelect ? sm.qs : p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
+        // queries: the copy made while scoring; attend-only launches make it
+        // here (the query is 4-byte aligned)
+        if constexpr (!kSelect) {
+            const uint32_t* qsrc = reinterpret_cast<const uint32_t*>(
+                p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD);
+            for (int i = tid; i < G * kD / 2; i += kThreads)
+                reinterpret_cast<uint32_t*>(sm.qs)[i] = qsrc[i];
+            __syncthreads();
+        }
+        const __nv_bfloat16* qg = sm.qs;
         uint32_t qa0[8], qa2[8], qa1[8], qa3[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
