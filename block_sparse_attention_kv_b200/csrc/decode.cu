@@ -462,7 +462,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 #endif
 
 template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM>
-__global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOCKS)
+__global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t smem_raw[];
@@ -867,18 +867,6 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
             __syncthreads();
         }
         const __nv_bfloat16* qg = sm.qs;
-        uint32_t qa0[8], qa2[8], qa1[8], qa3[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if constexpr (BIG_GROUP) {
-                qa0[j] = g < G ? ld_u32(qg + g * kD + 16 * j + 2 * t4) : 0u;
-                qa2[j] = g < G ? ld_u32(qg + g * kD + 16 * j + 8 + 2 * t4) : 0u;
-                qa1[j] = g + 8 < G ? ld_u32(qg + (g + 8) * kD + 16 * j + 2 * t4) : 0u;
-                qa3[j] = g + 8 < G ? ld_u32(qg + (g + 8) * kD + 16 * j + 8 + 2 * t4) : 0u;
-            } else {
-                qa0[j] = qa2[j] = qa1[j] = qa3[j] = 0u;  // unused (see the page loop)
-            }
-        }
         float o[16][4];
 #pragma unroll
         for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
@@ -969,15 +957,19 @@ __global__ void __launch_bounds__(kThreads, BIG_GROUP ? 1 : ABSP_DECODE_MIN_BLOC
                     const int ch = (j & 3) * 2 + (mi & 1);
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4(kh + tok * 128 + ((ch ^ ri) << 4), b0, b1, b2, b3);
+                    // the query fragments are re-read from shared memory at
+                    // each use rather than held through the page loop: no
+                    // kernel spills at 128 registers (two CTAs per SM)
+                    const uint32_t qx = g < G ? ld_u32(qg + g * kD + 16 * j + 2 * t4) : 0u;
+                    const uint32_t qy = g < G ? ld_u32(qg + g * kD + 16 * j + 8 + 2 * t4) : 0u;
                     if constexpr (BIG_GROUP) {
-                        mma_bf16(s0[0], s0[1], s0[2], s0[3], qa0[j], qa1[j], qa2[j], qa3[j], b0, b1);
-                        mma_bf16(s1[0], s1[1], s1[2], s1[3], qa0[j], qa1[j], qa2[j], qa3[j], b2, b3);
+                        const uint32_t qz =
+                            g + 8 < G ? ld_u32(qg + (g + 8) * kD + 16 * j + 2 * t4) : 0u;
+                        const uint32_t qw =
+                            g + 8 < G ? ld_u32(qg + (g + 8) * kD + 16 * j + 8 + 2 * t4) : 0u;
+                        mma_bf16(s0[0], s0[1], s0[2], s0[3], qx, qz, qy, qw, b0, b1);
+                        mma_bf16(s1[0], s1[1], s1[2], s1[3], qx, qz, qy, qw, b2, b3);
                     } else {
-                        // the query fragments are re-read at each use (from
-                        // shared memory in full mode): 16 fewer live
-                        // registers through the page loop, and no spills
-                        const uint32_t qx = g < G ? ld_u32(qg + g * kD + 16 * j + 2 * t4) : 0u;
-                        const uint32_t qy = g < G ? ld_u32(qg + g * kD + 16 * j + 8 + 2 * t4) : 0u;
                         mma_bf16_top(s0[0], s0[1], qx, qy, b0, b1);
                         mma_bf16_top(s1[0], s1[1], qx, qy, b2, b3);
                     }
