@@ -458,7 +458,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 }
 
 #ifndef ABSP_DECODE_MIN_BLOCKS
-#define ABSP_DECODE_MIN_BLOCKS 2
+#define ABSP_DECODE_MIN_BLOCKS 2  // CTAs per SM the register budget is built for
 #endif
 
 template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM>
@@ -1292,7 +1292,7 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     int C = pick_cluster(pairs, num_sms);
     cudaError_t e = cudaSuccess;
     for (; C >= 1; C /= 2) {
-        // region B: scores + select scratch, or this CTA's page slots, or the
+        // region B: scores + select scratch, or this CTA's page buffers, or the
         // warp merge; region A: code ring, or (CTA 0) the cluster merge
         size_t regB = 0, regA = 0, scratch = 0;
         if (do_select) {
