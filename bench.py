@@ -18,9 +18,9 @@ writes.  `variants.plain` is the same measurement with absp_decode_step
 
 value   = layer-steps/s over all ranks (weak scaling: every rank decodes its
           own layer stack, no collective on the data path);
-e2e     = the same through absp_decode_step_host with pinned host buffers
-          (the kernel reads each layer's query from host memory and writes
-          its output there, inside every layer-step);
+e2e     = the same through absp_decode_step_host_ex (same flags) with
+          pinned host buffers (the kernel reads each layer's query from host
+          memory and writes its output there, inside every layer-step);
 roofline= algorithmic bytes of a layer-step (centroid codes + per-channel
           parameters + valid selected K/V rows + q and out) / average launch
           time, against the measured HBM copy bandwidth;
@@ -553,12 +553,13 @@ def gpu_arm(args):
         q_host = [x.data.q.cpu().pin_memory() for x in layers]
         o_host = [torch.empty_like(q).pin_memory() for q in q_host]
         g2 = torch.cuda.CUDAGraph()
+        early = abi.ABSP_STEP_EARLY_PREFETCH                # as in the device graph
         for x, qh, oh in zip(layers, q_host, o_host):   # warm outside capture
-            abi.absp_decode_step_host(x.kv, x.cent, qh, x.budget, oh, x.ws, sc)
+            abi.absp_decode_step_host_ex(x.kv, x.cent, qh, x.budget, oh, x.ws, early, sc)
         stream.synchronize()
         with torch.cuda.graph(g2, stream=stream):
             for x, qh, oh in zip(layers, q_host, o_host):
-                abi.absp_decode_step_host(x.kv, x.cent, qh, x.budget, oh, x.ws, sc)
+                abi.absp_decode_step_host_ex(x.kv, x.cent, qh, x.budget, oh, x.ws, early, sc)
         with torch.cuda.stream(stream):
             ms_e2e = timed(g2, args.steps, args.warmup)
         for x, oh in zip(layers, o_host):

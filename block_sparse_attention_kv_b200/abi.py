@@ -108,6 +108,8 @@ def _load() -> ctypes.CDLL:
                                      c_void_p, c_void_p, c_size_t, c_uint32, c_void_p]),
         "absp_decode_step_host": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
+        "absp_decode_step_host_ex": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
+                                          c_void_p, c_void_p, c_size_t, c_uint32, c_void_p]),
         "absp_check_device_error": (st, [c_void_p, c_size_t, c_void_p, P(c_int32)]),
         "absp_build_quantize_noalloc": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p,
                                              c_void_p]),
@@ -130,6 +132,7 @@ EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_sizes_fm
             "absp_score_select_ex",
             "absp_sparse_decode",
             "absp_decode_step", "absp_decode_step_ex", "absp_decode_step_host",
+            "absp_decode_step_host_ex",
             "absp_check_device_error", "absp_build_quantize_noalloc",
             "absp_last_cuda_error", "absp_last_cuda_error_string")
 
@@ -345,6 +348,15 @@ def absp_decode_step_host(kv: LayerKV, cent: Centroids, q_host: torch.Tensor, bu
     _check(_lib.absp_decode_step_host(kv.ref, cent.ref, _ptr(q_host), int(budget),
                                       _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)),
            "absp_decode_step_host")
+
+
+def absp_decode_step_host_ex(kv: LayerKV, cent: Centroids, q_host: torch.Tensor, budget: int,
+                             out_host: torch.Tensor, ws: torch.Tensor, flags: int,
+                             stream=None) -> None:
+    _check(_lib.absp_decode_step_host_ex(kv.ref, cent.ref, _ptr(q_host), int(budget),
+                                         _ptr(out_host), _ptr(ws), ws.numel(), int(flags),
+                                         _stream(stream)),
+           "absp_decode_step_host_ex")
 
 
 def absp_build_quantize_noalloc(kv: LayerKV, cent: Centroids, device_status=None,

@@ -387,6 +387,15 @@ absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* 
 absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids* cent,
                                   const void* q_host, int32_t budget_tokens, void* out_host,
                                   void* ws, size_t ws_bytes, void* stream) {
+    return absp_decode_step_host_ex(kv, cent, q_host, budget_tokens, out_host, ws, ws_bytes, 0,
+                                    stream);
+}
+
+absp_status absp_decode_step_host_ex(const absp_layer_kv* kv, const absp_centroids* cent,
+                                     const void* q_host, int32_t budget_tokens, void* out_host,
+                                     void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
+    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX)) != 0)
+        return ABSP_ERR_INVALID_ARG;
     KvDesc d;
     absp_status st = make_desc(kv, &d, true);
     if (st != ABSP_OK) return st;
@@ -398,7 +407,7 @@ absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids*
     void* om = mapped_host(out_host);
     if (qm != nullptr && om != nullptr && aligned(qm, 4) && aligned(om, 4))
         return run_decode(kModeFull, kv, cent, qm, budget_tokens, nullptr, nullptr, om, ws,
-                          ws_bytes, stream);
+                          ws_bytes, stream, flags);
     const size_t act = static_cast<size_t>(d.S) * d.Hq * ABSP_HEAD_DIM * 2;
     uint8_t* qd = static_cast<uint8_t*>(ws) + kWsHeader;
     uint8_t* od = qd + round_up(act, kAlign);
@@ -406,7 +415,7 @@ absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids*
     cudaError_t e = cudaMemcpyAsync(qd, q_host, act, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return from_cuda(e);
     st = run_decode(kModeFull, kv, cent, qd, budget_tokens, nullptr, nullptr, od, ws, ws_bytes,
-                    stream);
+                    stream, flags);
     if (st != ABSP_OK) return st;
     e = cudaMemcpyAsync(out_host, od, act, cudaMemcpyDeviceToHost, s);
     return from_cuda(e);

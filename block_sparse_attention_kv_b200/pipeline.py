@@ -70,9 +70,13 @@ class DeviceLayer:
         else:
             abi.absp_decode_step(self.kv, self.cent, q, self.budget, out, self.ws, self.stream)
 
-    def decode_step_host(self, q_host, out_host):
-        abi.absp_decode_step_host(self.kv, self.cent, q_host, self.budget, out_host, self.ws,
-                                  self.stream)
+    def decode_step_host(self, q_host, out_host, flags: int = 0):
+        if flags:
+            abi.absp_decode_step_host_ex(self.kv, self.cent, q_host, self.budget, out_host,
+                                         self.ws, flags, self.stream)
+        else:
+            abi.absp_decode_step_host(self.kv, self.cent, q_host, self.budget, out_host,
+                                      self.ws, self.stream)
 
     # -- device-side faults ------------------------------------------------
     def check(self, ws=None):

@@ -255,6 +255,16 @@ ABSP_API absp_status absp_decode_step_host(const absp_layer_kv* kv,
                                   int32_t budget_tokens, void* out_host, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* absp_decode_step_host with the flags of absp_decode_step_ex
+ * (ABSP_STEP_EARLY_PREFETCH, ABSP_STEP_GROUP_MAX; other bits are rejected).
+ * With ABSP_STEP_EARLY_PREFETCH the cache-side reads (lengths, page table,
+ * centroid codes and parameters) start before the preceding launch on
+ * `stream` has completed; only the query is read after it. */
+ABSP_API absp_status absp_decode_step_host_ex(const absp_layer_kv* kv,
+                                     const absp_centroids* cent, const void* q_host,
+                                     int32_t budget_tokens, void* out_host, void* ws,
+                                     size_t ws_bytes, uint32_t flags, void* stream);
+
 /* Allocation-free steps 1-2.  The paper has no counterpart to this call;
  * it exists for callers that cannot allocate device memory where they build
  * a layer's centroids (code inside a framework that owns all device memory

@@ -140,6 +140,8 @@ def test_unknown_step_flags_rejected(abi):
     st = lib.absp_score_select_ex(kv.ref, None, None, 1024, None, None, None, 0,
                                   abi.ABSP_STEP_EARLY_PREFETCH, None)
     assert st == abi.ABSP_ERR_INVALID_ARG
+    st = lib.absp_decode_step_host_ex(kv.ref, None, None, 1024, None, None, 0, 0x80, None)
+    assert st == abi.ABSP_ERR_INVALID_ARG
 
 
 def test_null_layer_and_status_strings(abi):

@@ -249,14 +249,15 @@ def test_host_buffers_match_device_step(lib):
     # pinned (device-mapped: the kernel reads and writes them directly) and
     # pageable host buffers (copied through the workspace) give the same
     for pin in (True, False):
-        q_host = d.q.cpu()
-        out_host = torch.zeros_like(q_host)
-        if pin:
-            q_host, out_host = q_host.pin_memory(), out_host.pin_memory()
-        dl.decode_step_host(q_host, out_host)
-        torch.cuda.synchronize()
-        dl.check()
-        assert torch.equal(_bits(out_host), _bits(dl.out.cpu())), pin
+        for flags in (0, abi.ABSP_STEP_EARLY_PREFETCH):
+            q_host = d.q.cpu()
+            out_host = torch.zeros_like(q_host)
+            if pin:
+                q_host, out_host = q_host.pin_memory(), out_host.pin_memory()
+            dl.decode_step_host(q_host, out_host, flags=flags)
+            torch.cuda.synchronize()
+            dl.check()
+            assert torch.equal(_bits(out_host), _bits(dl.out.cpu())), (pin, flags)
 
 
 def test_repeated_steps_are_deterministic(lib):
