@@ -25,7 +25,8 @@ roofline= algorithmic bytes of a layer-step (centroid codes + per-channel
           parameters + valid selected K/V rows + q and out) / average launch
           time, against the measured HBM copy bandwidth;
 rebuild = centroid build + INT4 quantisation of every layer (steps 1-2),
-          timed separately (it runs once per cache, not per token);
+          timed separately (it runs once per cache, not per token); the
+          oracle's steps 1-2 are timed under cpu_baseline.rebuild;
 calibration = per-head normalised recall at block sizes 16/32/64 on a set of
           heads of varied concentration, and the block-size allocation it
           gives at the centroid memory of a uniform block size 32.
@@ -282,6 +283,33 @@ def time_oracle(prep, G, budget, steps: int = None, seconds: float = None):
     if lim is not None:
         lim.unregister() if hasattr(lim, "unregister") else None
     return done, el
+
+
+def time_oracle_rebuild(seconds: float):
+    """The oracle's steps 1-2 (centroids + INT4 codes) per KV head of the
+    workload's layer 0, 1 thread, for about `seconds`; returns (ms per layer
+    of Hkv heads, heads done)."""
+    from block_sparse_attention_kv_b200 import synth
+    from oracle import absp_oracle as O
+    w = synth.WORKLOADS[WORKLOAD]
+    hl = synth.host_layer(synth.make_layer(w, 0, "cpu"))
+    heads = [(O.head_keys_values(hl, 0, h)[0], int(hl.block_size[h]))
+             for h in range(len(hl.block_size))]
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except Exception:
+        lim = None
+    t0 = time.perf_counter()
+    done = 0
+    while done == 0 or time.perf_counter() - t0 < seconds:
+        keys, bs = heads[done % len(heads)]
+        O.quantize_centroids(O.build_centroids(keys, bs))
+        done += 1
+    el = time.perf_counter() - t0
+    if lim is not None and hasattr(lim, "unregister"):
+        lim.unregister()
+    return el / done * len(heads) * 1e3, done
 
 
 def _oracle_worker(task):
@@ -586,6 +614,11 @@ def gpu_arm(args):
                           f"{WORKLOAD} layer each, 1 thread each), {el2:.1f} s window"}
         except Exception as e:  # the single-thread figure above stands
             cpu["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+        ms, heads = time_oracle_rebuild(seconds=min(5.0, args.cpu_seconds))
+        cpu["rebuild"] = {
+            "ms_per_layer": ms, "cores": 1, "kind": "oracle",
+            "sample": f"{heads} (sequence, KV head) centroid builds + INT4 quantisations of "
+                      f"a {WORKLOAD} layer, numpy fp64, 1 thread (per layer: x Hkv)"}
 
     peak, peak_kind = hbm_peak()
     launch_ms = ms / (args.steps * L)
