@@ -1183,6 +1183,15 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
     if (e != cudaSuccess) return e;
     const bool cached = dev >= 0 && dev < kCacheDevices;
     int fit = -1;
+    // the one-time set-up below may run while the caller captures `st` into
+    // a graph: relaxed capture mode lets these calls (which touch no stream)
+    // through without disturbing the capture
+    cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+    cudaThreadExchangeStreamCaptureMode(&mode);
+    struct RestoreMode {
+        cudaStreamCaptureMode* m;
+        ~RestoreMode() { cudaThreadExchangeStreamCaptureMode(m); }
+    } restore{&mode};
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!cached || !configured[dev]) {
@@ -1214,7 +1223,9 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
         // an answer: it is not cached and the launch below reports the error
         std::lock_guard<std::mutex> lock(mu);
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess) {
+        cudaLaunchConfig_t q = cfg;   // the query needs no stream
+        q.stream = nullptr;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &q) == cudaSuccess) {
             fit = nclusters > 0 ? 1 : 0;
             if (cached) shapes[dev].insert(C, smem, fit);
         } else {
