@@ -614,15 +614,20 @@ def gpu_arm(args):
                           f"{WORKLOAD} layer each, 1 thread each), {el2:.1f} s window"}
         except Exception as e:  # the single-thread figure above stands
             cpu["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
-        ms, heads = time_oracle_rebuild(seconds=min(5.0, args.cpu_seconds))
+        rb_ms, heads = time_oracle_rebuild(seconds=min(5.0, args.cpu_seconds))
         cpu["rebuild"] = {
-            "ms_per_layer": ms, "cores": 1, "kind": "oracle",
+            "ms_per_layer": rb_ms, "cores": 1, "kind": "oracle",
             "sample": f"{heads} (sequence, KV head) centroid builds + INT4 quantisations of "
                       f"a {WORKLOAD} layer, numpy fp64, 1 thread (per layer: x Hkv)"}
 
     peak, peak_kind = hbm_peak()
     launch_ms = ms / (args.steps * L)
     achieved = bytes_per_launch / (launch_ms * 1e-3) / 1e9
+    # a launch cannot move its bytes much faster than a plain copy: a figure
+    # far above the copy peak means the timed region did not do the work
+    if achieved > 1.5 * peak:
+        raise RuntimeError(f"implausible launch time {launch_ms * 1e3:.2f} us "
+                           f"({achieved:.0f} GB/s for {bytes_per_launch:.0f} B)")
     traffic = recorded_traffic()
     line = {
         "metric": METRIC,
