@@ -72,6 +72,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--workloads", action="store_true",
+                    help="also time the fused step on the batched and long-context "
+                         "workloads (reported under 'workloads')")
     return ap.parse_args()
 
 
@@ -234,6 +237,52 @@ def rebuild_large(dev, stream, abi, pipeline, synth):
     torch.cuda.empty_cache()
     return {"workload": "rebuild_8x128k: 8 sequences x 131072 tokens, 8 KV heads",
             "ms": ms, "bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9}
+
+
+# layers per timed graph for the other workloads: enough distinct caches
+# that a replay never finds its inputs in L2 (every layer here is > 0.5 GB)
+OTHER_WORKLOADS = (("qwen3_8b_128k_36l", 4), ("batch32_32k_8l", 2), ("ragged64_paged", 2))
+
+
+def other_workloads(dev, stream, abi, pipeline, synth, timed, steps, warmup, peak):
+    """The fused early-prefetch step on the batched and long-context
+    workloads: per layer-step time and algorithmic bytes, same method as the
+    headline (CUDA graph over distinct layer caches, CUDA events)."""
+    out = {}
+    sc = stream.cuda_stream
+    flags = abi.ABSP_STEP_EARLY_PREFETCH
+    for name, nl in OTHER_WORKLOADS:
+        w = synth.WORKLOADS[name]
+        ys, nb = [], []
+        with torch.cuda.stream(stream):
+            for i in range(nl):
+                y = pipeline.DeviceLayer(synth.make_layer(w, i, dev), stream=sc)
+                y.build_centroids()
+                y.score_select()
+                stream.synchronize()
+                nb.append(step_bytes(y.data, y.sel.cpu().numpy(), y.sel_count.cpu().numpy()))
+                abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws,
+                                        flags, sc)
+                ys.append(y)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for y in ys:
+                abi.absp_decode_step_ex(y.kv, y.cent, y.data.q, y.budget, y.out, y.ws,
+                                        flags, sc)
+        with torch.cuda.stream(stream):
+            ms = timed(g, steps, warmup)
+        for y in ys:
+            y.check()
+        us = ms / (steps * nl) * 1e3
+        bpl = float(np.mean(nb))
+        gbs = bpl / (us * 1e-6) / 1e9
+        out[name] = {"us_per_layer_step": us, "layers": nl, "bytes_per_launch": bpl,
+                     "achieved_gbs": gbs, "frac": gbs / peak,
+                     "sequences": w.num_seqs, "budget": w.budget}
+        del g, ys
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------- CPU oracle leg --
@@ -576,6 +625,11 @@ def gpu_arm(args):
             del gv, vl
         del fws
 
+    extra = None
+    if args.workloads:
+        extra = other_workloads(dev, stream, abi, pipeline, synth, timed,
+                                args.steps, args.warmup, hbm_peak()[0])
+
     e2e = None
     if not args.no_e2e:
         q_host = [x.data.q.cpu().pin_memory() for x in layers]
@@ -674,6 +728,8 @@ def gpu_arm(args):
                     "large": None if rb_large is None else
                     {**rb_large, "frac": rb_large["achieved_gbs"] / peak}},
     }
+    if extra is not None:
+        line["workloads"] = extra
     del g
     if rank == 0:
         print(json.dumps(line), flush=True)
