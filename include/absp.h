@@ -27,6 +27,11 @@
  *     are recorded in the first bytes of the workspace and reported by
  *     absp_check_device_error(); kernels never trap.
  *   - head_dim must be 128 and page_size 16 (ABSP_ERR_UNSUPPORTED otherwise).
+ *   - Calls that only launch work on `stream` may be captured into a CUDA
+ *     graph, in any capture mode, including the first launch of a kernel in
+ *     the process (its one-time set-up never touches the capturing
+ *     stream).  Not capturable: absp_check_device_error (it waits for the
+ *     stream) and the first absp_build_quantize_noalloc call per device.
  *   - No call throws; every call returns an absp_status.
  */
 #ifndef ABSP_H_
