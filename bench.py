@@ -55,6 +55,9 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn decode layer-steps/s at 32K ctx; achieved HBM GB/s vs B200 peak"
 UNIT = "layer-steps/s"
 WORKLOAD = "llama31_8b_32k"
+WORKLOAD_DESC = (f"{WORKLOAD}: Llama-3.1-8B-shaped attention layer decode, 32 q / 8 kv "
+                 f"heads, head_dim 128, batch 1, ctx 32768, budget 2048 tokens, "
+                 f"block sizes per kv head from {{16,32,64}}, INT4 centroids")
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "block_sparse_attention_kv_b200", "csrc", f)
@@ -408,7 +411,8 @@ def reference_arm(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / max(done, 1) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "step": "one (sequence, KV head) decode unit"},
+            "config": {"workload": WORKLOAD_DESC, "step": "one (sequence, KV head) decode unit",
+                       "parallelism": "one host thread (rank 0 only)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -697,9 +701,7 @@ def gpu_arm(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": (f"{WORKLOAD}: Llama-3.1-8B-shaped attention layer decode, 32 q / 8 kv "
-                         f"heads, head_dim 128, batch 1, ctx 32768, budget 2048 tokens, "
-                         f"block sizes per kv head from {{16,32,64}}, INT4 centroids"),
+            "workload": WORKLOAD_DESC,
             "layers_per_step": L,
             "step": f"one decode token through {L} layers with distinct caches",
             "l2": f"inputs larger than L2: {L} distinct layer caches (~{L * 128 // 1024} GiB)",
