@@ -368,7 +368,9 @@ def _oracle_worker(task):
     """One process of the all-cores oracle timing: (units done, seconds)."""
     seconds, head, barrier = task
     prep, G, budget = oracle_layer_sample(0, heads=[head])
-    barrier.wait()                      # every worker times the same window
+    # every worker times the same window; a worker that never arrives
+    # breaks the barrier for the others instead of holding them forever
+    barrier.wait(timeout=300)
     return time_oracle(prep, G, budget, seconds=seconds)
 
 
