@@ -154,6 +154,49 @@ def _ptr(t) -> int:
     return t.data_ptr()
 
 
+def _bad(what: str, msg: str):
+    raise AbspError(ABSP_ERR_INVALID_ARG, f"{what}: {msg}")
+
+
+def _arg(t, what: str, name: str, dtype=None, numel: int = 0, where: str = "cuda"):
+    """Address of tensor argument `name` of call `what`, after checking what
+    the C ABI assumes of the buffer behind it and cannot check itself: its
+    element type, a dense row-major layout, its memory space ("cuda": the
+    current device; "host": host memory) and at least `numel` elements.
+    A raw integer address or None passes through unchecked."""
+    if t is None or isinstance(t, int):
+        return t
+    if not isinstance(t, torch.Tensor):
+        _bad(what, f"{name} must be a torch.Tensor or an address")
+    if dtype is not None and t.dtype != dtype:
+        _bad(what, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        _bad(what, f"{name} must be contiguous")
+    if where == "cuda":
+        if not t.is_cuda:
+            _bad(what, f"{name} must be in device memory")
+        if t.device.index != torch.cuda.current_device():
+            _bad(what, f"{name} is on cuda:{t.device.index}, the current device is "
+                       f"cuda:{torch.cuda.current_device()}")
+    elif t.is_cuda:
+        _bad(what, f"{name} must be in host memory")
+    if t.numel() < numel:
+        _bad(what, f"{name} holds {t.numel()} elements, {numel} needed")
+    return t.data_ptr()
+
+
+def _ws(ws, what: str):
+    """(address, bytes) of a device workspace tensor."""
+    if not isinstance(ws, torch.Tensor):
+        _bad(what, "ws must be a device tensor")
+    return _arg(ws, what, "ws"), ws.numel() * ws.element_size()
+
+
+def _qo(kv: "LayerKV") -> int:
+    """Elements of a query or output buffer: [S][Hq][128]."""
+    return kv.c.num_seqs * kv.c.num_q_heads * HEAD_DIM
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
@@ -286,91 +329,139 @@ def absp_select_capacity(kv: LayerKV, budget: int) -> int:
 
 
 def absp_workspace_init(ws: torch.Tensor, stream=None) -> None:
-    _check(_lib.absp_workspace_init(_ptr(ws), ws.numel(), _stream(stream)),
-           "absp_workspace_init")
+    w, wb = _ws(ws, "absp_workspace_init")
+    _check(_lib.absp_workspace_init(w, wb, _stream(stream)), "absp_workspace_init")
+
+
+def _cent(kv: LayerKV, cent: Centroids, what: str):
+    """cent.ref after checking its buffers against the layer's sizes."""
+    cb, sb, zb = absp_centroid_sizes_fmt(kv, cent.format)
+    _arg(cent.codes, what, "codes", torch.uint8, cb)
+    if cent.format == ABSP_CENTROIDS_INT4:
+        _arg(cent.scale, what, "scale", torch.float32, sb // 4)
+        _arg(cent.zp, what, "zp", torch.int32, zb // 4)
+    return cent.ref
+
+
+def _sel(kv: LayerKV, sel, sel_count, budget: int, what: str):
+    n = kv.c.num_seqs * kv.c.num_kv_heads
+    kmax = absp_select_capacity(kv, budget) if isinstance(sel, torch.Tensor) else 0
+    return (_arg(sel, what, "sel", torch.int32, n * kmax),
+            _arg(sel_count, what, "sel_count", torch.int32, n))
 
 
 def absp_build_centroids(kv: LayerKV, ws: torch.Tensor, stream=None) -> None:
-    _check(_lib.absp_build_centroids(kv.ref, _ptr(ws), ws.numel(), _stream(stream)),
-           "absp_build_centroids")
+    w, wb = _ws(ws, "absp_build_centroids")
+    _check(_lib.absp_build_centroids(kv.ref, w, wb, _stream(stream)), "absp_build_centroids")
 
 
 def absp_quantize_centroids(kv: LayerKV, ws: torch.Tensor, cent: Centroids, stream=None) -> None:
-    _check(_lib.absp_quantize_centroids(kv.ref, _ptr(ws), ws.numel(), cent.ref,
-                                        _stream(stream)), "absp_quantize_centroids")
+    what = "absp_quantize_centroids"
+    w, wb = _ws(ws, what)
+    _check(_lib.absp_quantize_centroids(kv.ref, w, wb, _cent(kv, cent, what), _stream(stream)),
+           what)
 
 
 def absp_score_select(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
                       sel: torch.Tensor, sel_count: torch.Tensor, ws: torch.Tensor,
                       stream=None) -> None:
-    _check(_lib.absp_score_select(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(sel),
-                                  _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
-           "absp_score_select")
+    what = "absp_score_select"
+    w, wb = _ws(ws, what)
+    sp, cp = _sel(kv, sel, sel_count, budget, what)
+    _check(_lib.absp_score_select(kv.ref, _cent(kv, cent, what),
+                                  _arg(q, what, "q", torch.bfloat16, _qo(kv)), int(budget),
+                                  sp, cp, w, wb, _stream(stream)), what)
 
 
 def absp_append_centroids(kv: LayerKV, cent: Centroids, exceeded, ws: torch.Tensor,
                           stream=None) -> None:
-    _check(_lib.absp_append_centroids(kv.ref, cent.ref, _ptr(exceeded), _ptr(ws), ws.numel(),
-                                      _stream(stream)), "absp_append_centroids")
+    what = "absp_append_centroids"
+    w, wb = _ws(ws, what)
+    ex = _arg(exceeded, what, "exceeded", torch.int32, kv.c.num_seqs * kv.c.num_kv_heads)
+    _check(_lib.absp_append_centroids(kv.ref, _cent(kv, cent, what), ex, w, wb,
+                                      _stream(stream)), what)
 
 
 def absp_score_select_ex(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
                          sel: torch.Tensor, sel_count: torch.Tensor, ws: torch.Tensor,
                          flags: int, stream=None) -> None:
-    _check(_lib.absp_score_select_ex(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(sel),
-                                     _ptr(sel_count), _ptr(ws), ws.numel(), int(flags),
-                                     _stream(stream)), "absp_score_select_ex")
+    what = "absp_score_select_ex"
+    w, wb = _ws(ws, what)
+    sp, cp = _sel(kv, sel, sel_count, budget, what)
+    _check(_lib.absp_score_select_ex(kv.ref, _cent(kv, cent, what),
+                                     _arg(q, what, "q", torch.bfloat16, _qo(kv)), int(budget),
+                                     sp, cp, w, wb, int(flags), _stream(stream)), what)
 
 
 def absp_sparse_decode(kv: LayerKV, q: torch.Tensor, sel: torch.Tensor,
                        sel_count: torch.Tensor, budget: int, out: torch.Tensor,
                        ws: torch.Tensor, stream=None) -> None:
-    _check(_lib.absp_sparse_decode(kv.ref, _ptr(q), _ptr(sel), _ptr(sel_count), int(budget),
-                                   _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
-           "absp_sparse_decode")
+    what = "absp_sparse_decode"
+    w, wb = _ws(ws, what)
+    sp, cp = _sel(kv, sel, sel_count, budget, what)
+    _check(_lib.absp_sparse_decode(kv.ref, _arg(q, what, "q", torch.bfloat16, _qo(kv)), sp, cp,
+                                   int(budget), _arg(out, what, "out", torch.bfloat16, _qo(kv)),
+                                   w, wb, _stream(stream)), what)
 
 
 def absp_decode_step(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
                      out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
-    _check(_lib.absp_decode_step(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(out), _ptr(ws),
-                                 ws.numel(), _stream(stream)), "absp_decode_step")
+    what = "absp_decode_step"
+    w, wb = _ws(ws, what)
+    _check(_lib.absp_decode_step(kv.ref, _cent(kv, cent, what),
+                                 _arg(q, what, "q", torch.bfloat16, _qo(kv)), int(budget),
+                                 _arg(out, what, "out", torch.bfloat16, _qo(kv)), w, wb,
+                                 _stream(stream)), what)
 
 
 def absp_decode_step_ex(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,
                         out: torch.Tensor, ws: torch.Tensor, flags: int, stream=None) -> None:
-    _check(_lib.absp_decode_step_ex(kv.ref, cent.ref, _ptr(q), int(budget), _ptr(out), _ptr(ws),
-                                    ws.numel(), int(flags), _stream(stream)),
-           "absp_decode_step_ex")
+    what = "absp_decode_step_ex"
+    w, wb = _ws(ws, what)
+    _check(_lib.absp_decode_step_ex(kv.ref, _cent(kv, cent, what),
+                                    _arg(q, what, "q", torch.bfloat16, _qo(kv)), int(budget),
+                                    _arg(out, what, "out", torch.bfloat16, _qo(kv)), w, wb,
+                                    int(flags), _stream(stream)), what)
 
 
 def absp_decode_step_host(kv: LayerKV, cent: Centroids, q_host: torch.Tensor, budget: int,
                           out_host: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
-    _check(_lib.absp_decode_step_host(kv.ref, cent.ref, _ptr(q_host), int(budget),
-                                      _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)),
-           "absp_decode_step_host")
+    what = "absp_decode_step_host"
+    w, wb = _ws(ws, what)
+    _check(_lib.absp_decode_step_host(
+        kv.ref, _cent(kv, cent, what),
+        _arg(q_host, what, "q_host", torch.bfloat16, _qo(kv), where="host"), int(budget),
+        _arg(out_host, what, "out_host", torch.bfloat16, _qo(kv), where="host"), w, wb,
+        _stream(stream)), what)
 
 
 def absp_decode_step_host_ex(kv: LayerKV, cent: Centroids, q_host: torch.Tensor, budget: int,
                              out_host: torch.Tensor, ws: torch.Tensor, flags: int,
                              stream=None) -> None:
-    _check(_lib.absp_decode_step_host_ex(kv.ref, cent.ref, _ptr(q_host), int(budget),
-                                         _ptr(out_host), _ptr(ws), ws.numel(), int(flags),
-                                         _stream(stream)),
-           "absp_decode_step_host_ex")
+    what = "absp_decode_step_host_ex"
+    w, wb = _ws(ws, what)
+    _check(_lib.absp_decode_step_host_ex(
+        kv.ref, _cent(kv, cent, what),
+        _arg(q_host, what, "q_host", torch.bfloat16, _qo(kv), where="host"), int(budget),
+        _arg(out_host, what, "out_host", torch.bfloat16, _qo(kv), where="host"), w, wb,
+        int(flags), _stream(stream)), what)
 
 
 def absp_build_quantize_noalloc(kv: LayerKV, cent: Centroids, device_status=None,
                                 stream=None) -> None:
     """Centroid build + INT4 quantisation without a caller workspace (the
     library's static scratch array is used instead)."""
-    _check(_lib.absp_build_quantize_noalloc(kv.ref, cent.ref, _ptr(device_status),
-                                            _stream(stream)), "absp_build_quantize_noalloc")
+    what = "absp_build_quantize_noalloc"
+    _check(_lib.absp_build_quantize_noalloc(
+        kv.ref, _cent(kv, cent, what),
+        _arg(device_status, what, "device_status", torch.int32, 2), _stream(stream)), what)
 
 
 def absp_check_device_error(ws: torch.Tensor, stream=None):
     """Returns (status, detail); status is ABSP_OK when no device fault."""
     d = c_int32()
-    st = _lib.absp_check_device_error(_ptr(ws), ws.numel(), _stream(stream), ctypes.byref(d))
+    w, wb = _ws(ws, "absp_check_device_error")
+    st = _lib.absp_check_device_error(w, wb, _stream(stream), ctypes.byref(d))
     if st == ABSP_ERR_CUDA or st == ABSP_ERR_INVALID_ARG:
         raise AbspError(st, "absp_check_device_error")
     return st, d.value

@@ -111,9 +111,10 @@ def test_invalid_layers_are_rejected(abi, over, status):
 
 def test_misaligned_pages_rejected_by_decode_calls(abi):
     kv = _kv(abi, k_pages=0x100010)
-    with pytest.raises(abi.AbspError) as e:
-        abi.absp_build_centroids(kv, torch.zeros(1 << 20, dtype=torch.uint8))
-    assert e.value.status == abi.ABSP_ERR_INVALID_ARG
+    # a fake, aligned and large enough workspace address: only the page
+    # alignment can fail
+    st = abi.lib().absp_build_centroids(kv.ref, 0x400000, 1 << 20, None)
+    assert st == abi.ABSP_ERR_INVALID_ARG
 
 
 def test_budget_limits(abi):
@@ -126,10 +127,41 @@ def test_budget_limits(abi):
 
 def test_small_workspace_rejected_before_launch(abi):
     kv = _kv(abi)
-    tiny = torch.zeros(64, dtype=torch.uint8)
+    st = abi.lib().absp_build_centroids(kv.ref, 0x400000, 64, None)
+    assert st == abi.ABSP_ERR_INVALID_ARG
+
+
+def test_binding_checks_tensor_arguments(abi):
+    # what the C ABI cannot see behind a raw pointer is checked by the
+    # binding before the call: element type, dense layout, memory space and
+    # element count; raw addresses pass through unchecked
+    q = torch.zeros((2, 8, 128), dtype=torch.bfloat16)
+    assert abi._arg(q, "f", "q", torch.bfloat16, q.numel(), where="host") == q.data_ptr()
+    assert abi._arg(0x1000, "f", "q", torch.bfloat16, 1 << 30) == 0x1000
+    assert abi._arg(None, "f", "q", torch.bfloat16, 1) is None
+    cases = [
+        (dict(t=q.float()), "bfloat16"),
+        (dict(t=q.transpose(0, 1)), "contiguous"),
+        (dict(t=q, numel=q.numel() + 1), "elements"),
+        (dict(t=q, where="cuda"), "device memory"),
+        (dict(t=[1, 2]), "torch.Tensor"),
+    ]
+    for kw, text in cases:
+        args = dict(dtype=torch.bfloat16, numel=q.numel(), where="host")
+        args.update(kw)
+        t = args.pop("t")
+        with pytest.raises(abi.AbspError) as e:
+            abi._arg(t, "f", "q", **args)
+        assert e.value.status == abi.ABSP_ERR_INVALID_ARG
+        assert text in str(e.value) and "q" in str(e.value)
+
+
+def test_public_calls_refuse_host_tensors_for_device_buffers(abi):
+    kv = _kv(abi)
     with pytest.raises(abi.AbspError) as e:
-        abi.absp_build_centroids(kv, tiny)
+        abi.absp_build_centroids(kv, torch.zeros(1 << 20, dtype=torch.uint8))
     assert e.value.status == abi.ABSP_ERR_INVALID_ARG
+    assert "ws must be in device memory" in str(e.value)
 
 
 def test_unknown_step_flags_rejected(abi):
