@@ -35,8 +35,10 @@ absp_status absp::make_desc(const absp_layer_kv* kv, KvDesc* d, bool need_v) {
     if (kv->num_q_heads / kv->num_kv_heads > ABSP_MAX_GROUP) return ABSP_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(kv->max_pages_per_seq) * ABSP_PAGE_SIZE > (1ll << 30))
         return ABSP_ERR_UNSUPPORTED;
-    // tensor-map row coordinates are int32
-    if (kv->num_phys_pages * kv->num_kv_heads * ABSP_PAGE_SIZE >= (1ll << 31))
+    // tensor-map row coordinates are int32 (the first test keeps the
+    // product below from overflowing)
+    if (kv->num_phys_pages >= (1ll << 31) ||
+        kv->num_phys_pages * kv->num_kv_heads * ABSP_PAGE_SIZE >= (1ll << 31))
         return ABSP_ERR_UNSUPPORTED;
     if (kv->seq_lens == nullptr || kv->page_table == nullptr || kv->k_pages == nullptr ||
         kv->block_size == nullptr || (need_v && kv->v_pages == nullptr))

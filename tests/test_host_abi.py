@@ -101,6 +101,8 @@ def test_sizes_follow_the_layout(abi):
     (dict(num_q_heads=2 * 17), 2),          # group of 17 > 16
     (dict(k_pages=0x100010), 1),            # not 256-byte aligned
     (dict(seq_lens=0), 1),
+    (dict(num_phys_pages=1 << 27), 2),      # 2^27 pages x 2 heads x 16 rows = 2^32
+    (dict(num_phys_pages=1 << 60), 2),      # would wrap the row count
 ])
 def test_invalid_layers_are_rejected(abi, over, status):
     kv = _kv(abi, **over)
