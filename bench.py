@@ -244,7 +244,8 @@ def rebuild_large(dev, stream, abi, pipeline, synth):
 
 # layers per timed graph for the other workloads: enough distinct caches
 # that a replay never finds its inputs in L2 (every layer here is > 0.5 GB)
-OTHER_WORKLOADS = (("qwen3_8b_128k_36l", 4), ("batch32_32k_8l", 2), ("ragged64_paged", 2))
+OTHER_WORKLOADS = (("qwen3_8b_128k_36l", 4), ("batch32_32k_8l", 2), ("ragged64_paged", 2),
+                   ("gqa16_batch96_16k", 2))
 
 
 def other_workloads(dev, stream, abi, pipeline, synth, timed, steps, warmup, peak):

@@ -92,6 +92,11 @@ WORKLOADS = {
     "ragged64_paged": Workload("ragged64_paged", layers=1, num_seqs=64,
                                num_q_heads=32, num_kv_heads=8,
                                ragged=(4096, 65536), budget=2048, seed=1004),
+    # GQA 16 batch: 96 sequences x 16K, 32 query heads over 2 KV heads
+    # (block sizes 16 and 64), the widest group the kernels take.
+    "gqa16_batch96_16k": Workload("gqa16_batch96_16k", layers=1, num_seqs=96,
+                                  num_q_heads=32, num_kv_heads=2, ctx=16384,
+                                  budget=1024, block_sizes=(16, 64), seed=1007),
     # Full centroid rebuild + INT4 quantisation at batch 8 x 131072.
     "rebuild_8x128k": Workload("rebuild_8x128k", layers=1, num_seqs=8,
                                num_q_heads=32, num_kv_heads=8, ctx=131072,

@@ -39,6 +39,10 @@ def test_block_size_mix_and_named_shapes():
     p = synth.plan_layer(w, 0)
     assert p.max_pages == 32768 // 16 and p.num_phys_pages == 2048
     assert synth.WORKLOADS["tiny_8k"].block_sizes == (16, 64)
+    g = synth.plan_layer(synth.WORKLOADS["gqa16_batch96_16k"], 0)
+    assert g.seq_lens.shape == (96,) and np.all(g.seq_lens == 16384)
+    assert g.block_size.tolist() == [16, 64]
+    assert synth.WORKLOADS["gqa16_batch96_16k"].num_q_heads // 2 == 16
 
 
 def test_ragged_lengths_log_uniform_range():
