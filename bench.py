@@ -295,10 +295,15 @@ def oracle_layer_sample(layer_index: int = 0, heads=None):
     """Host copy of one layer plus the oracle's prebuilt centroids (of the
     KV heads in `heads`, all when None)."""
     from block_sparse_attention_kv_b200 import synth
-    from oracle import absp_oracle as O
     w = synth.WORKLOADS[WORKLOAD]
     d = synth.make_layer(w, layer_index, "cpu")
-    hl = synth.host_layer(d)
+    return _oracle_prep(synth.host_layer(d), heads)
+
+
+def _oracle_prep(hl, heads=None):
+    """(units, G, budget) of a host layer: one unit per (sequence, KV head),
+    each with the oracle's prebuilt dequantised centroids."""
+    from oracle import absp_oracle as O
     prep = []
     for s in range(hl.q_bits.shape[0]):
         qf = O.decode_bf16(hl.q_bits[s])
@@ -311,6 +316,44 @@ def oracle_layer_sample(layer_index: int = 0, heads=None):
             prep.append((qf, h, chat, keys, vals, bs, int(hl.seq_lens[s])))
     G = hl.q_bits.shape[1] // len(hl.block_size)
     return prep, G, int(hl.budget)
+
+
+def oracle_workload_sample(name: str, k: int = 4):
+    """A bounded host sample of workload `name` for the oracle: k of its
+    sequences (evenly spaced in its sorted length list, so a ragged batch is
+    covered from short to long), generated as a small layer with the same
+    head counts, block sizes and budget.  Returns (prep, G, budget, lengths,
+    units per layer-step of the whole workload)."""
+    from block_sparse_attention_kv_b200 import synth
+    w = synth.WORKLOADS[name]
+    lens = np.sort(synth.draw_seq_lens(w))
+    k = min(k, len(lens))
+    pick = [int(lens[(2 * i + 1) * len(lens) // (2 * k)]) for i in range(k)]
+    bs = [int(b) for b in synth.draw_block_sizes(w, 0)]
+    sw = synth.custom(f"{name}_sample", k, w.num_q_heads, w.num_kv_heads, pick, bs,
+                      w.budget, seed=w.seed)
+    prep, G, budget = _oracle_prep(synth.host_layer(synth.make_layer(sw, 0, "cpu")))
+    return prep, G, budget, pick, w.num_seqs * w.num_kv_heads
+
+
+def oracle_workloads(seconds: float) -> dict:
+    """The oracle's steps 3-5 on a bounded sample of each of the other
+    workloads, 1 thread, about `seconds` each; the layer-step time is the
+    mean time of a sampled (sequence, KV head) unit times the workload's
+    units per layer-step."""
+    out = {}
+    for name, _ in OTHER_WORKLOADS:
+        prep, G, budget, pick, units = oracle_workload_sample(name)
+        time_oracle(prep, G, budget, steps=1)                    # warm
+        done, el = time_oracle(prep, G, budget, seconds=seconds)
+        ms = el / done * units * 1e3
+        out[name] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_layer_step": ms, "cores": 1,
+                     "kind": "oracle",
+                     "sample": f"{done} (sequence, KV head) units of {len(pick)} sequences "
+                               f"(lengths {pick}) generated with the workload's head counts, "
+                               f"block sizes and budget; mean unit time x {units} units "
+                               f"per layer-step; numpy fp64, 1 thread, {el:.1f} s"}
+    return out
 
 
 def time_oracle(prep, G, budget, steps: int = None, seconds: float = None):
@@ -420,6 +463,8 @@ def reference_arm(args):
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+    if args.workloads:
+        line["workloads"] = oracle_workloads(min(3.0, args.cpu_seconds))
     print(json.dumps(line), flush=True)
 
 
@@ -636,6 +681,9 @@ def gpu_arm(args):
     if args.workloads:
         extra = other_workloads(dev, stream, abi, pipeline, synth, timed,
                                 args.steps, args.warmup, hbm_peak()[0])
+        if rank == 0 and not args.no_cpu_baseline:
+            for name, cb in oracle_workloads(min(3.0, args.cpu_seconds)).items():
+                extra[name]["cpu_baseline"] = cb
 
     e2e = None
     if not args.no_e2e:
