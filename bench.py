@@ -318,6 +318,14 @@ def _oracle_prep(hl, heads=None):
     return prep, G, int(hl.budget)
 
 
+def sample_lengths(lens, k: int) -> list:
+    """k lengths evenly spaced through the sorted `lens` (the midpoints of k
+    equal slices of the sorted list)."""
+    lens = np.sort(np.asarray(lens))
+    k = min(k, len(lens))
+    return [int(lens[(2 * i + 1) * len(lens) // (2 * k)]) for i in range(k)]
+
+
 def oracle_workload_sample(name: str, k: int = 4):
     """A bounded host sample of workload `name` for the oracle: k of its
     sequences (evenly spaced in its sorted length list, so a ragged batch is
@@ -326,9 +334,8 @@ def oracle_workload_sample(name: str, k: int = 4):
     units per layer-step of the whole workload)."""
     from block_sparse_attention_kv_b200 import synth
     w = synth.WORKLOADS[name]
-    lens = np.sort(synth.draw_seq_lens(w))
-    k = min(k, len(lens))
-    pick = [int(lens[(2 * i + 1) * len(lens) // (2 * k)]) for i in range(k)]
+    pick = sample_lengths(synth.draw_seq_lens(w), k)
+    k = len(pick)
     bs = [int(b) for b in synth.draw_block_sizes(w, 0)]
     sw = synth.custom(f"{name}_sample", k, w.num_q_heads, w.num_kv_heads, pick, bs,
                       w.budget, seed=w.seed)

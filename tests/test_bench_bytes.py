@@ -90,3 +90,20 @@ def test_llama31_8b_32k_mean_over_the_benchmarks_64_layers():
     w = synth.WORKLOADS["llama31_8b_32k"]
     mean = np.mean([_full_length_closed_form(w, l) for l in bench.rank_layer_ids(0, 64)])
     assert mean == 8_935_424
+
+
+def test_oracle_sample_lengths_span_a_ragged_batch():
+    lens = np.arange(1, 65) * 1000
+    assert bench.sample_lengths(lens, 4) == [9000, 25000, 41000, 57000]
+    assert bench.sample_lengths([5, 3], 4) == [3, 5]
+    w = synth.WORKLOADS["ragged64_paged"]
+    pick = bench.sample_lengths(synth.draw_seq_lens(w), 4)
+    assert pick == sorted(pick) and set(pick) <= set(synth.draw_seq_lens(w).tolist())
+
+
+def test_oracle_workload_sample_keeps_the_workload_shape():
+    prep, G, budget, pick, units = bench.oracle_workload_sample("gqa16_batch96_16k", k=2)
+    w = synth.WORKLOADS["gqa16_batch96_16k"]
+    assert G == 16 and budget == w.budget and units == 96 * 2
+    assert pick == [16384, 16384] and len(prep) == 2 * 2
+    assert sorted({u[5] for u in prep}) == [16, 64]          # the per-head block sizes
