@@ -8,7 +8,6 @@ import ctypes
 import os
 import re
 
-import numpy as np
 import pytest
 import torch
 
