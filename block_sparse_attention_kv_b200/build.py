@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libabsp.so")
 SOURCES = ["abi.cu", "centroids.cu", "decode.cu", "noalloc.cu"]
-HEADERS = ["absp_internal.cuh"]
+HEADERS = ["absp_internal.cuh", "absp_trace.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

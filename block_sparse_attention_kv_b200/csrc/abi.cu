@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "absp_internal.cuh"
+#include "absp_trace.h"
 
 using namespace absp;
 
@@ -312,12 +313,14 @@ absp_status absp_select_capacity(const absp_layer_kv* kv, int32_t budget_tokens,
 }
 
 absp_status absp_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    ABSP_TRACE("absp_workspace_init");
     if (ws == nullptr || ws_bytes < static_cast<size_t>(kWsHeader) || !aligned(ws, kAlign))
         return ABSP_ERR_INVALID_ARG;
     return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 absp_status absp_build_centroids(const absp_layer_kv* kv, void* ws, size_t ws_bytes, void* stream) {
+    ABSP_TRACE("absp_build_centroids");
     KvDesc d;
     absp_status st = make_desc(kv, &d, false);
     if (st != ABSP_OK) return st;
@@ -327,6 +330,7 @@ absp_status absp_build_centroids(const absp_layer_kv* kv, void* ws, size_t ws_by
 
 absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws, size_t ws_bytes,
                                     const absp_centroids* out, void* stream) {
+    ABSP_TRACE("absp_quantize_centroids");
     KvDesc d;
     absp_status st = make_desc(kv, &d, false);
     if (st != ABSP_OK) return st;
@@ -338,6 +342,7 @@ absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws, size_t ws
 
 absp_status absp_append_centroids(const absp_layer_kv* kv, const absp_centroids* cent,
                                   int32_t* exceeded, void* ws, size_t ws_bytes, void* stream) {
+    ABSP_TRACE("absp_append_centroids");
     KvDesc d;
     absp_status st = make_desc(kv, &d, false);
     if (st != ABSP_OK) return st;
@@ -351,6 +356,7 @@ absp_status absp_append_centroids(const absp_layer_kv* kv, const absp_centroids*
 absp_status absp_score_select(const absp_layer_kv* kv, const absp_centroids* cent, const void* q,
                               int32_t budget_tokens, int32_t* sel, int32_t* sel_count, void* ws,
                               size_t ws_bytes, void* stream) {
+    ABSP_TRACE("absp_score_select");
     return run_decode(kModeSelect, kv, cent, q, budget_tokens, sel, sel_count, nullptr, ws,
                       ws_bytes, stream);
 }
@@ -358,6 +364,7 @@ absp_status absp_score_select(const absp_layer_kv* kv, const absp_centroids* cen
 absp_status absp_sparse_decode(const absp_layer_kv* kv, const void* q, const int32_t* sel,
                                const int32_t* sel_count, int32_t budget_tokens, void* out,
                                void* ws, size_t ws_bytes, void* stream) {
+    ABSP_TRACE("absp_sparse_decode");
     return run_decode(kModeAttend, kv, nullptr, q, budget_tokens, const_cast<int32_t*>(sel),
                       const_cast<int32_t*>(sel_count), out, ws, ws_bytes, stream);
 }
@@ -365,6 +372,7 @@ absp_status absp_sparse_decode(const absp_layer_kv* kv, const void* q, const int
 absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centroids* cent, const void* q,
                              int32_t budget_tokens, void* out, void* ws, size_t ws_bytes,
                              void* stream) {
+    ABSP_TRACE("absp_decode_step");
     return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
                       stream);
 }
@@ -372,6 +380,7 @@ absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centroids* cent
 absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                 const void* q, int32_t budget_tokens, void* out, void* ws,
                                 size_t ws_bytes, uint32_t flags, void* stream) {
+    ABSP_TRACE("absp_decode_step_ex");
     if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX)) != 0)
         return ABSP_ERR_INVALID_ARG;
     return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
@@ -381,6 +390,7 @@ absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* c
 absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* cent, const void* q,
                                  int32_t budget_tokens, int32_t* sel, int32_t* sel_count,
                                  void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
+    ABSP_TRACE("absp_score_select_ex");
     if ((flags & ~static_cast<uint32_t>(ABSP_STEP_GROUP_MAX)) != 0) return ABSP_ERR_INVALID_ARG;
     return run_decode(kModeSelect, kv, cent, q, budget_tokens, sel, sel_count, nullptr, ws,
                       ws_bytes, stream, flags);
@@ -389,6 +399,7 @@ absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* 
 absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids* cent,
                                   const void* q_host, int32_t budget_tokens, void* out_host,
                                   void* ws, size_t ws_bytes, void* stream) {
+    ABSP_TRACE("absp_decode_step_host");
     return absp_decode_step_host_ex(kv, cent, q_host, budget_tokens, out_host, ws, ws_bytes, 0,
                                     stream);
 }
@@ -396,6 +407,7 @@ absp_status absp_decode_step_host(const absp_layer_kv* kv, const absp_centroids*
 absp_status absp_decode_step_host_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                      const void* q_host, int32_t budget_tokens, void* out_host,
                                      void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
+    ABSP_TRACE("absp_decode_step_host_ex");
     if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX)) != 0)
         return ABSP_ERR_INVALID_ARG;
     KvDesc d;
@@ -424,6 +436,7 @@ absp_status absp_decode_step_host_ex(const absp_layer_kv* kv, const absp_centroi
 }
 
 absp_status absp_check_device_error(void* ws, size_t ws_bytes, void* stream, int32_t* detail) {
+    ABSP_TRACE("absp_check_device_error");
     if (ws == nullptr || ws_bytes < static_cast<size_t>(kWsHeader)) return ABSP_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t word[2] = {0, 0};

@@ -20,6 +20,7 @@
 #include <mutex>
 
 #include "absp_internal.cuh"
+#include "absp_trace.h"
 
 namespace {
 
@@ -53,6 +54,7 @@ cudaError_t noalloc_scratch(void** out) {
 extern "C" absp_status absp_build_quantize_noalloc(const absp_layer_kv* kv,
                                                    const absp_centroids* out,
                                                    int32_t* device_status, void* stream) {
+    ABSP_TRACE("absp_build_quantize_noalloc");
     absp::KvDesc d;
     absp_status st = absp::make_desc(kv, &d, false);
     if (st != ABSP_OK) return st;
