@@ -14,6 +14,9 @@ Per (sequence, KV head) of a layer:
   reports top-K page recall above 0.9 in every layer of Llama-3.1-8B for
   asymmetric per-channel INT4 centroids;
 * the same for BF16 centroids (the page's Fig. 13 precision baseline);
+* planted recall: the share of the planted q-aligned tokens inside the
+  selected blocks (1.0 expected: they are what the generator makes
+  relevant);
 * token recall: the share of the exact top-budget tokens (by the group-summed
   query's dot product with each key) that lie in the selected blocks.  On
   i.i.d. synthetic keys a block mean cannot single out isolated tokens, so
@@ -47,6 +50,20 @@ def token_recall(layer, s: int, h: int, sel, bs: int) -> float:
     top = np.lexsort((np.arange(dots.shape[0]), -dots))[:B]
     toks = set(O.selected_tokens(np.asarray(sel), bs, keys.shape[0]).tolist())
     return float(np.mean([int(t) in toks for t in top]))
+
+
+def planted_recall(layer, planted_mask) -> float:
+    """Share of the planted q-aligned tokens (planted_mask(s, h) -> bool mask
+    over the sequence) inside the oracle's INT4 selection, over all
+    (sequence, KV head) of the layer."""
+    res = O.run_layer(layer, with_attention=False)
+    hit = tot = 0
+    for (s, h), hr in res.heads.items():
+        m = np.asarray(planted_mask(s, h), dtype=bool)
+        toks = O.selected_tokens(hr.sel, hr.block_size, hr.seq_len)
+        tot += int(m.sum())
+        hit += int(m[toks].sum())
+    return hit / tot if tot else 1.0
 
 
 def layer_diagnostics(layer) -> dict:

@@ -32,3 +32,10 @@ def test_int4_page_recall_on_the_llama_shaped_layer():
     assert int4 > 0.9                      # Fig. 8's bar, on synthetic keys
     assert bf16 >= int4
     assert all(v["int4_page_recall"] > 0.8 for v in d.values())
+
+
+def test_planted_spans_are_recalled_on_configs_0_to_2():
+    for name, layer in (("tiny_8k", 0), ("llama31_8b_32k", 0), ("qwen3_8b_128k_36l", 35)):
+        d = synth.make_layer(synth.WORKLOADS[name], layer, "cpu")
+        hl = synth.host_layer(d)
+        assert D.planted_recall(hl, lambda s, h: synth.planted_mask(d.plan, s, h)) == 1.0, name
