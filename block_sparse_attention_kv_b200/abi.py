@@ -82,6 +82,7 @@ def _load() -> ctypes.CDLL:
     P = POINTER
     sig = {
         "absp_status_string": (c_char_p, [st]),
+        "absp_build_id": (c_char_p, []),
         "absp_centroid_sizes": (st, [P(absp_layer_kv), P(c_size_t), P(c_size_t), P(c_size_t)]),
         "absp_centroid_sizes_fmt": (st, [P(absp_layer_kv), c_int32, P(c_size_t), P(c_size_t),
                                          P(c_size_t)]),
@@ -124,7 +125,7 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("absp_status_string", "absp_centroid_sizes", "absp_centroid_sizes_fmt",
+EXPORTED = ("absp_status_string", "absp_build_id", "absp_centroid_sizes", "absp_centroid_sizes_fmt",
             "absp_centroid_row_offset",
             "absp_build_workspace_size", "absp_decode_workspace_size",
             "absp_select_capacity", "absp_workspace_init", "absp_build_centroids",
@@ -277,6 +278,11 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 def absp_status_string(status: int) -> str:
     return _lib.absp_status_string(int(status)).decode()
+
+
+def absp_build_id() -> str:
+    """Source hash the loaded library was compiled from."""
+    return _lib.absp_build_id().decode()
 
 
 def absp_last_cuda_error() -> int:

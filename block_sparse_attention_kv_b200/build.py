@@ -3,13 +3,16 @@
     python -m block_sparse_attention_kv_b200.build [--verbose-ptxas]
 
 The shared library lands in block_sparse_attention_kv_b200/lib/ and is what
-the ctypes binding loads.  cudart is linked statically, so the library only
+the ctypes binding loads.  A library is reused only when it was built from
+the current sources: the hash of the sources, headers, this script and the
+flags is compiled into it (absp_build_id()) and kept beside it.  cudart is linked statically, so the library only
 needs the CUDA driver at run time.
 """
 
 from __future__ import annotations
 
 import argparse
+import hashlib
 import os
 import shutil
 import subprocess
@@ -24,7 +27,10 @@ LIB = os.path.join(LIBDIR, "libabsp.so")
 SOURCES = ["abi.cu", "centroids.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["absp_internal.cuh", "absp_trace.h"]
 
+STAMP = LIB + ".build_id"
+
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17"]
 
 
 def nvcc() -> str:
@@ -34,23 +40,45 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found (set NVCC or install the CUDA toolkit)")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
+def source_hash() -> str:
+    """SHA-256 (first 16 hex digits) of everything the library is built
+    from: the CUDA sources and headers, the public header, this script and
+    the compile flags.  It is compiled into the library (absp_build_id) and
+    decides whether an existing library is reused."""
+    h = hashlib.sha256()
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(INCLUDE, "absp.h"))
     deps.append(os.path.abspath(__file__))
-    return any(os.path.getmtime(p) > t for p in deps)
+    for p in deps:
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(ARCH + FLAGS).encode())
+    return h.hexdigest()[:16]
+
+
+def built_id() -> str:
+    """Build id recorded beside the library at its last build ('' if none)."""
+    try:
+        with open(STAMP) as f:
+            return f.read().strip()
+    except OSError:
+        return ""
+
+
+def _stale(want: str) -> bool:
+    return not os.path.exists(LIB) or built_id() != want
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile the library if any source is newer than it; return its path."""
-    if not force and not verbose_ptxas and not _stale():
+    """Compile the library unless the one in place was built from exactly
+    the current sources (same source hash); return its path."""
+    want = source_hash()
+    if not force and not verbose_ptxas and not _stale(want):
         return LIB
     os.makedirs(LIBDIR, exist_ok=True)
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
+    cmd = [nvcc(), *ARCH, *FLAGS, f"-DABSP_BUILD_ID=\"{want}\"", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", INCLUDE, "-cudart", "static",
            "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES]
@@ -69,6 +97,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if verbose_ptxas:
         sys.stderr.write(res.stderr)
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(want + "\n")
     return LIB
 
 

@@ -451,6 +451,12 @@ absp_status absp_check_device_error(void* ws, size_t ws_bytes, void* stream, int
     return word[0] == ABSP_ERR_TIMEOUT ? ABSP_ERR_TIMEOUT : ABSP_ERR_DEVICE_FAULT;
 }
 
+#ifndef ABSP_BUILD_ID
+#define ABSP_BUILD_ID "unknown"
+#endif
+
+const char* absp_build_id(void) { return ABSP_BUILD_ID; }
+
 int absp_last_cuda_error(void) { return t_last_cuda; }
 
 const char* absp_last_cuda_error_string(void) {

@@ -10,9 +10,12 @@
 // and the centroid buffers (outputs).
 //
 // The scratch is a file-scope __device__ array of ABSP_NOALLOC_BUILD_WS_BYTES
-// bytes.  It lives in this file's own module: every GPU on which the module
-// is loaded (at the first call of the entry point on that GPU) holds it until
-// the process exits.  All calls on one GPU share it and it keeps the last
+// bytes.  It lives in the library's module: every GPU on which the module is
+// loaded holds it until the process exits.  With lazy module loading (the
+// CUDA default) that is from the first call of the entry point on that GPU;
+// with eager loading (CUDA_MODULE_LOADING=EAGER) it is from the creation of
+// the context on every GPU the process uses, whether or not the entry point
+// is ever called.  All calls on one GPU share it and it keeps the last
 // call's contents, so each call clears the parts that must start at zero
 // (the error word and the per-channel min/max keys), and calls whose work
 // overlaps on the GPU (different streams, no ordering between them) race on
@@ -29,21 +32,61 @@ __device__ __align__(256) uint8_t g_noalloc_build_ws[ABSP_NOALLOC_BUILD_WS_BYTES
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_ws_ptr[kMaxDevices] = {};
+unsigned long long g_ctx_id[kMaxDevices] = {};  // context the address belongs to
+
+// Driver entry points that identify the current context (resolved once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+struct CtxFns {
+    CtxGetCurrentFn current = nullptr;
+    CtxGetIdFn id = nullptr;
+};
+const CtxFns& ctx_fns() {
+    static const CtxFns f = [] {
+        CtxFns r;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            r.current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            r.id = reinterpret_cast<CtxGetIdFn>(p);
+        return r;
+    }();
+    return f;
+}
+
+// Unique id of the calling thread's current context, 0 if none or unknown.
+unsigned long long current_ctx_id() {
+    const CtxFns& f = ctx_fns();
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (f.current == nullptr || f.id == nullptr || f.current(&c) != CUDA_SUCCESS || c == nullptr)
+        return 0;
+    return f.id(c, &id) == CUDA_SUCCESS ? id : 0;
+}
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// with cudaGetSymbolAddress, once per device, with that device current.
+// with cudaGetSymbolAddress, once per device and context, with that device
+// current.  The lookup is repeated when the device's context is not the one
+// the cached address belongs to (a cudaDeviceReset destroys the primary
+// context, and the array is reloaded at another address in the next one).
 cudaError_t noalloc_scratch(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (g_ws_ptr[dev] == nullptr) {
+    const unsigned long long ctx = current_ctx_id();
+    if (g_ws_ptr[dev] == nullptr || ctx == 0 || ctx != g_ctx_id[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_build_ws);
         if (e != cudaSuccess) return e;
         g_ws_ptr[dev] = p;
+        // the lookup made the device's context current if none was
+        g_ctx_id[dev] = current_ctx_id();
     }
     *out = g_ws_ptr[dev];
     return cudaSuccess;

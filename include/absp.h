@@ -114,6 +114,13 @@ typedef struct absp_centroids {
 /* Human-readable name of a status code (static string, never NULL). */
 ABSP_API const char* absp_status_string(absp_status status);
 
+/* Identity of the sources this library was compiled from: the first 16 hex
+ * digits of a SHA-256 over its CUDA sources, headers, build script and
+ * compile flags ("unknown" for a build that did not define it).  Static
+ * string, host only, never fails.  The paper has no counterpart: it lets a
+ * record of a run name the exact sources that ran. */
+ABSP_API const char* absp_build_id(void);
+
 /* Bytes of the three centroid buffers for `kv` (host only, no launch). */
 ABSP_API absp_status absp_centroid_sizes(const absp_layer_kv* kv, size_t* codes_bytes,
                                 size_t* scale_bytes, size_t* zp_bytes);
@@ -281,11 +288,14 @@ ABSP_API absp_status absp_decode_step_host_ex(const absp_layer_kv* kv,
  *   - Layers whose absp_build_workspace_size exceeds that size are
  *     rejected with ABSP_ERR_UNSUPPORTED before anything is launched.
  *   - No device memory is allocated by the call.  The array itself is held
- *     on every GPU where the library's static-scratch module is loaded (at
- *     the first call on that GPU) until the process exits.
+ *     on every GPU where the library's module is loaded, until the process
+ *     exits: from the first call on that GPU under lazy module loading (the
+ *     CUDA default), from context creation on every GPU the process uses
+ *     under CUDA_MODULE_LOADING=EAGER.
  *   - The first call on each device looks the array's device address up on
- *     the host (with that device current); make that first call before any
- *     stream capture.
+ *     the host (with that device current), and so does the first call after
+ *     the device's context changed (after a cudaDeviceReset, say); make such
+ *     a call before any stream capture.
  *   - All calls on a GPU share the array; each call clears what must start
  *     at zero.  Calls whose GPU work can overlap (unordered streams) race on
  *     the array and must be ordered by the caller.

@@ -183,3 +183,11 @@ def test_null_layer_and_status_strings(abi):
     assert abi.absp_status_string(0) == "ok"
     assert "bounds" in abi.absp_status_string(abi.ABSP_ERR_DEVICE_FAULT)
     assert abi.absp_status_string(99) == "unknown status"
+
+
+def test_build_id_names_the_current_sources(abi):
+    # build() reuses a library only when it was compiled from the current
+    # sources, and the library carries that source hash
+    assert abi.LIB_PATH == absp_build.LIB or os.environ.get("ABSP_LIB")
+    assert abi.absp_build_id() == absp_build.source_hash()
+    assert absp_build.built_id() == absp_build.source_hash()
