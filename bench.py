@@ -75,9 +75,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
-    ap.add_argument("--workloads", action="store_true",
-                    help="also time the fused step on the batched and long-context "
-                         "workloads (reported under 'workloads')")
+    ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the long-context and batched workloads (reported "
+                         "under 'workloads')")
     return ap.parse_args()
 
 
@@ -191,6 +192,17 @@ def rebuild_bytes(d):
 
 # ---------------------------------------------------------------- ranks --
 
+def bench_config(layers: int, world: int) -> dict:
+    """The workload description both arms report."""
+    return {
+        "workload": WORKLOAD_DESC,
+        "layers_per_step": layers,
+        "step": f"one decode token through {layers} layers with distinct caches",
+        "l2": f"inputs larger than L2: {layers} distinct layer caches (~{layers * 128 // 1024} GiB)",
+        "parallelism": f"dp{world} (independent layer stacks per GPU)",
+    }
+
+
 def rank_layer_ids(rank: int, layers: int) -> list:
     """Layer seeds of one rank: every rank decodes its own layer stack."""
     return [rank * layers + i for i in range(layers)]
@@ -220,16 +232,14 @@ def rebuild_large(dev, stream, abi, pipeline, synth):
     ws = abi.alloc_workspace(abi.absp_build_workspace_size(y.kv), dev)
     sc = stream.cuda_stream
     for _ in range(2):
-        abi.absp_build_centroids(y.kv, ws, sc)
-        abi.absp_quantize_centroids(y.kv, ws, y.cent, sc)
+        abi.absp_build_quantize_centroids(y.kv, ws, y.cent, sc)
     stream.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     reps = 5
     e0.record(stream)
     for _ in range(reps):
-        abi.absp_build_centroids(y.kv, ws, sc)
-        abi.absp_quantize_centroids(y.kv, ws, y.cent, sc)
+        abi.absp_build_quantize_centroids(y.kv, ws, y.cent, sc)
     e1.record(stream)
     stream.synchronize()
     st, _ = abi.absp_check_device_error(ws, sc)
@@ -242,22 +252,30 @@ def rebuild_large(dev, stream, abi, pipeline, synth):
             "ms": ms, "bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9}
 
 
-# layers per timed graph for the other workloads: enough distinct caches
-# that a replay never finds its inputs in L2 (every layer here is > 0.5 GB)
-OTHER_WORKLOADS = (("qwen3_8b_128k_36l", 4), ("batch32_32k_8l", 2), ("ragged64_paged", 2),
-                   ("gqa16_batch96_16k", 2))
+# The other workloads, each at the layer count it is stated with; a timed
+# graph replays every layer once per step, so the layer-steps of one replay
+# read far more than L2 holds (selected K/V + codes per replay: Qwen3 128K
+# 36 x ~19 MB, batch 32 8 x ~144 MB, ragged 64 2 x ~0.6 GB, GQA 16 4 x
+# ~0.1 GB).  The ragged batch is one layer of 64 sequences; two distinct
+# caches keep a replay from finding the previous one in L2.
+OTHER_WORKLOADS = (("qwen3_8b_128k_36l", 36), ("batch32_32k_8l", 8), ("ragged64_paged", 2),
+                   ("gqa16_batch96_16k", 4))
 
 
-def other_workloads(dev, stream, abi, pipeline, synth, timed, steps, warmup, peak):
-    """The fused early-prefetch step on the batched and long-context
+def other_workloads(dev, stream, abi, pipeline, synth, timed, steps, warmup, peak,
+                    parity: bool = True):
+    """The fused early-prefetch step on the long-context and batched
     workloads: per layer-step time and algorithmic bytes, same method as the
-    headline (CUDA graph over distinct layer caches, CUDA events)."""
+    headline (CUDA graph over distinct layer caches, CUDA events), and a
+    parity record of the oracle on one of the timed layers (two sequences of
+    a batch)."""
     out = {}
     sc = stream.cuda_stream
     flags = abi.ABSP_STEP_EARLY_PREFETCH
     for name, nl in OTHER_WORKLOADS:
         w = synth.WORKLOADS[name]
         ys, nb = [], []
+        t_gen = time.perf_counter()
         with torch.cuda.stream(stream):
             for i in range(nl):
                 y = pipeline.DeviceLayer(synth.make_layer(w, i, dev), stream=sc)
@@ -269,6 +287,7 @@ def other_workloads(dev, stream, abi, pipeline, synth, timed, steps, warmup, pea
                                         flags, sc)
                 ys.append(y)
         stream.synchronize()
+        t_gen = time.perf_counter() - t_gen
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for y in ys:
@@ -281,9 +300,17 @@ def other_workloads(dev, stream, abi, pipeline, synth, timed, steps, warmup, pea
         us = ms / (steps * nl) * 1e3
         bpl = float(np.mean(nb))
         gbs = bpl / (us * 1e-6) / 1e9
-        out[name] = {"us_per_layer_step": us, "layers": nl, "bytes_per_launch": bpl,
-                     "achieved_gbs": gbs, "frac": gbs / peak,
-                     "sequences": w.num_seqs, "budget": w.budget}
+        rec = {"us_per_layer_step": us, "layers": nl, "bytes_per_launch": bpl,
+               "achieved_gbs": gbs, "frac": gbs / peak, "value": 1e6 / us,
+               "unit": UNIT, "sequences": w.num_seqs, "kv_heads": w.num_kv_heads,
+               "q_heads": w.num_q_heads, "budget": w.budget,
+               "ctx": w.ctx if w.ragged is None else f"log-uniform {list(w.ragged)}",
+               "setup_s": t_gen}
+        if parity:
+            S = ys[0].data.num_seqs
+            seqs = [0] if S == 1 else [0, S - 1]
+            rec["parity"] = parity_record(ys[0], name, seqs)
+        out[name] = rec
         del g, ys
         torch.cuda.empty_cache()
     return out
@@ -493,13 +520,14 @@ def reference_arm(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / max(done, 1) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD_DESC, "step": "one (sequence, KV head) decode unit",
-                       "parallelism": "one host thread (rank 0 only)"},
+            "config": bench_config(args.layers, args.gpus),
+            "launch": "the CPU oracle (numpy fp64), one host thread, rank 0 only; each step "
+                      "one (sequence, KV head) unit of a layer-step",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
-    if args.workloads:
+    if not args.no_workloads:
         line["workloads"] = oracle_workloads(min(3.0, args.cpu_seconds))
     print(json.dumps(line), flush=True)
 
@@ -535,6 +563,52 @@ def calibration_summary(dev, synth):
     }
 
 
+# ------------------------------------------------------ parity record --
+
+def parity_record(x, name: str, seqs=None) -> dict:
+    """The oracle against the library on one layer that the timed region
+    decoded, checked after it: INT4 codes, scales and zero points exact,
+    selections exact up to counted boundary near-ties, and the output that
+    the timed launches left in x.out within the tolerances of the oracle
+    run on the library's own selection, for every KV head of the sampled
+    sequences."""
+    from block_sparse_attention_kv_b200 import synth
+    from oracle import absp_oracle as O
+    from oracle import parity as PR
+    d = x.data
+    S, Hkv = d.num_seqs, d.num_kv_heads
+    seqs = list(range(S)) if seqs is None else list(seqs)
+    t0 = time.perf_counter()
+    x.score_select()                  # the selection the fused launches made
+    torch.cuda.synchronize()
+    x.check()
+    hl = synth.host_layer(d, seqs)
+    hl.budget = x.budget
+    sel = x.sel.cpu().numpy()
+    cnt = x.sel_count.cpu().numpy()
+    over = {(i, h): sel[s, h, :cnt[s, h]] for i, s in enumerate(seqs) for h in range(Hkv)}
+    res = O.run_layer(hl, sel_override=over)
+    rep = PR.Report()
+    for i, s in enumerate(seqs):
+        for h in range(Hkv):
+            hr = res.heads[(i, h)]
+            rep.heads += 1
+            n = hr.centroids.shape[0]
+            scale, zp = x.params_of(s, h)
+            PR.compare_codes(rep, hr, x.codes_of(s, h, n).cpu().numpy(),
+                             scale.cpu().numpy(), zp.cpu().numpy())
+            PR.compare_selection(rep, hr, sel[s, h, :cnt[s, h]])
+    out = x.out[torch.as_tensor(seqs, device=x.out.device)].float().cpu().numpy()
+    PR.compare_outputs(rep, out, res.out)
+    return {"workload": name, "sequences": seqs, "kv_heads": rep.heads,
+            "code_mismatch": rep.code_mismatch, "param_mismatch": rep.param_mismatch,
+            "sel_mismatch": rep.sel_mismatch, "near_ties": rep.near_ties,
+            "out_max_abs": rep.out_max_abs, "out_mean_abs": rep.out_mean_abs,
+            "tolerance": {"out_max_abs": PR.OUT_MAX_ABS, "out_mean_abs": PR.OUT_MEAN_ABS,
+                          "tie_rel": PR.TIE_REL},
+            "ok": rep.ok(), "seconds": time.perf_counter() - t0}
+
+
 # ----------------------------------------------------------- GPU arm --
 
 def gpu_arm(args):
@@ -568,24 +642,35 @@ def gpu_arm(args):
             layers.append(pipeline.DeviceLayer(d, stream=stream.cuda_stream))
     stream.synchronize()
 
-    # steps 1-2 for every layer, timed (once per cache)
+    # steps 1-2 for every layer, timed (once per cache): the one-call build
+    # (absp_build_quantize_centroids, one fused launch per layer here), and
+    # the two separate calls
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ws_n = max(abi.absp_build_workspace_size(x.kv) for x in layers)
     bws = abi.alloc_workspace(ws_n, dev)
     sc = stream.cuda_stream
-    for x in layers[:2]:                               # warm-up
-        abi.absp_build_centroids(x.kv, bws, sc)
-        abi.absp_quantize_centroids(x.kv, bws, x.cent, sc)
-    stream.synchronize()
-    ev0.record(stream)
-    for x in layers:
-        abi.absp_build_centroids(x.kv, bws, sc)
-        abi.absp_quantize_centroids(x.kv, bws, x.cent, sc)
-    ev1.record(stream)
-    stream.synchronize()
-    rebuild_ms = ev0.elapsed_time(ev1) / L
-    st, _ = abi.absp_check_device_error(bws, sc)
-    assert st == abi.ABSP_OK, "device fault while building centroids"
+
+    def time_builds(fused: bool) -> float:
+        def one(x):
+            if fused:
+                abi.absp_build_quantize_centroids(x.kv, bws, x.cent, sc)
+            else:
+                abi.absp_build_centroids(x.kv, bws, sc)
+                abi.absp_quantize_centroids(x.kv, bws, x.cent, sc)
+        for x in layers[:2]:                           # warm-up
+            one(x)
+        stream.synchronize()
+        ev0.record(stream)
+        for x in layers:
+            one(x)
+        ev1.record(stream)
+        stream.synchronize()
+        st, _ = abi.absp_check_device_error(bws, sc)
+        assert st == abi.ABSP_OK, "device fault while building centroids"
+        return ev0.elapsed_time(ev1) / L
+
+    rebuild_two_ms = time_builds(False)
+    rebuild_ms = time_builds(True)
     rb_bytes = sum(rebuild_bytes(x.data) for x in layers) / L
     del bws
     rb_large = None if args.no_variants else rebuild_large(dev, stream, abi, pipeline, synth)
@@ -646,6 +731,10 @@ def gpu_arm(args):
     for x in layers:
         x.check()
     del g_plain
+    # the headline layer 0 against the oracle, after its timed launches
+    parity = None
+    if not args.no_parity and rank == 0:
+        parity = parity_record(layers[0], WORKLOAD)
 
     # incremental tail-row update (one launch per layer); with unchanged
     # lengths it rewrites every tail row with the same bytes
@@ -714,9 +803,10 @@ def gpu_arm(args):
         del fws
 
     extra = None
-    if args.workloads:
+    if not args.no_workloads:
         extra = other_workloads(dev, stream, abi, pipeline, synth, timed,
-                                args.steps, args.warmup, hbm_peak()[0])
+                                args.steps, args.warmup, hbm_peak()[0],
+                                parity=not args.no_parity)
         if rank == 0 and not args.no_cpu_baseline:
             for name, cb in oracle_workloads(min(3.0, args.cpu_seconds)).items():
                 extra[name]["cpu_baseline"] = cb
@@ -805,21 +895,16 @@ def gpu_arm(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": WORKLOAD_DESC,
-            "layers_per_step": L,
-            "step": f"one decode token through {L} layers with distinct caches",
-            "l2": f"inputs larger than L2: {L} distinct layer caches (~{L * 128 // 1024} GiB)",
-            "launch": "CUDA graph of fused score/select/attend launches, PDL, "
-                      "ABSP_STEP_EARLY_PREFETCH",
-            "parallelism": f"dp{world} (independent layer stacks per GPU)",
-        },
+        "config": bench_config(L, world),
+        "launch": "CUDA graph of fused score/select/attend launches, PDL, "
+                  "ABSP_STEP_EARLY_PREFETCH",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} HBM copy bandwidth",
                      "kernel": "decode_kernel<full>",
                      "bytes_per_launch": bytes_per_launch, "launch_us": launch_ms * 1e3},
         "cpu_baseline": cpu,
+        "parity": parity,
         "e2e": e2e,
         "gpu_launches": L * args.steps,
         "variants": {**fixed, "plain": {"value": aggregate_rate(world, L, args.steps, ms_plain),
@@ -833,6 +918,10 @@ def gpu_arm(args):
         "rebuild": {"ms_per_layer": rebuild_ms, "bytes_per_layer": rb_bytes,
                     "achieved_gbs": rb_bytes / (rebuild_ms * 1e-3) / 1e9,
                     "frac": rb_bytes / (rebuild_ms * 1e-3) / 1e9 / peak,
+                    "call": "absp_build_quantize_centroids",
+                    "two_calls": {"ms_per_layer": rebuild_two_ms,
+                                  "frac": rb_bytes / (rebuild_two_ms * 1e-3) / 1e9 / peak,
+                                  "call": "absp_build_centroids + absp_quantize_centroids"},
                     "large": None if rb_large is None else
                     {**rb_large, "frac": rb_large["achieved_gbs"] / peak}},
     }

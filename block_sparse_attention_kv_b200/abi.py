@@ -28,6 +28,7 @@ ABSP_ERR_TIMEOUT = 5
 
 ABSP_STEP_EARLY_PREFETCH = 1
 ABSP_STEP_GROUP_MAX = 2
+ABSP_STEP_DIAG_WAIT_TIMEOUT = 0x100
 ABSP_CENTROIDS_INT4 = 0
 ABSP_CENTROIDS_BF16 = 1
 
@@ -96,6 +97,8 @@ def _load() -> ctypes.CDLL:
                                          P(absp_centroids), c_void_p]),
         "absp_score_select": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
                                    c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+        "absp_build_quantize_centroids": (st, [P(absp_layer_kv), c_void_p, c_size_t,
+                                               P(absp_centroids), c_void_p]),
         "absp_append_centroids": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_void_p,
                                        c_size_t, c_void_p]),
         "absp_score_select_ex": (st, [P(absp_layer_kv), P(absp_centroids), c_void_p, c_int32,
@@ -129,7 +132,8 @@ EXPORTED = ("absp_status_string", "absp_build_id", "absp_centroid_sizes", "absp_
             "absp_centroid_row_offset",
             "absp_build_workspace_size", "absp_decode_workspace_size",
             "absp_select_capacity", "absp_workspace_init", "absp_build_centroids",
-            "absp_quantize_centroids", "absp_append_centroids", "absp_score_select",
+            "absp_quantize_centroids", "absp_build_quantize_centroids",
+            "absp_append_centroids", "absp_score_select",
             "absp_score_select_ex",
             "absp_sparse_decode",
             "absp_decode_step", "absp_decode_step_ex", "absp_decode_step_host",
@@ -366,6 +370,14 @@ def absp_quantize_centroids(kv: LayerKV, ws: torch.Tensor, cent: Centroids, stre
     w, wb = _ws(ws, what)
     _check(_lib.absp_quantize_centroids(kv.ref, w, wb, _cent(kv, cent, what), _stream(stream)),
            what)
+
+
+def absp_build_quantize_centroids(kv: LayerKV, ws: torch.Tensor, cent: Centroids,
+                                  stream=None) -> None:
+    what = "absp_build_quantize_centroids"
+    w, wb = _ws(ws, what)
+    _check(_lib.absp_build_quantize_centroids(kv.ref, w, wb, _cent(kv, cent, what),
+                                              _stream(stream)), what)
 
 
 def absp_score_select(kv: LayerKV, cent: Centroids, q: torch.Tensor, budget: int,

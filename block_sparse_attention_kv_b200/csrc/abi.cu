@@ -216,6 +216,10 @@ absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* 
     a.zp = cent ? cent->zp : nullptr;
     a.cfmt = cent ? cent->format : ABSP_CENTROIDS_INT4;
     a.group_max = (flags & ABSP_STEP_GROUP_MAX) != 0 ? 1 : 0;
+    a.diag_timeout = (flags & ABSP_STEP_DIAG_WAIT_TIMEOUT) != 0 ? 1 : 0;
+    if (a.diag_timeout && (mode == kModeAttend || a.group_max || a.cfmt != ABSP_CENTROIDS_INT4 ||
+                           d.G > 8 || (flags & ABSP_STEP_EARLY_PREFETCH) != 0))
+        return ABSP_ERR_UNSUPPORTED;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.out = static_cast<__nv_bfloat16*>(out);
     a.sel = sel;
@@ -340,6 +344,19 @@ absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws, size_t ws
                                      out->format, static_cast<cudaStream_t>(stream)));
 }
 
+absp_status absp_build_quantize_centroids(const absp_layer_kv* kv, void* ws, size_t ws_bytes,
+                                          const absp_centroids* out, void* stream) {
+    ABSP_TRACE("absp_build_quantize_centroids");
+    KvDesc d;
+    absp_status st = make_desc(kv, &d, false);
+    if (st != ABSP_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, build_ws_bytes(d))) != ABSP_OK) return st;
+    if ((st = check_cent(out)) != ABSP_OK) return st;
+    return from_cuda(launch_build_quantize(d, build_ws_layout(ws, d), out->codes, out->scale,
+                                           out->zp, out->format,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 absp_status absp_append_centroids(const absp_layer_kv* kv, const absp_centroids* cent,
                                   int32_t* exceeded, void* ws, size_t ws_bytes, void* stream) {
     ABSP_TRACE("absp_append_centroids");
@@ -381,7 +398,8 @@ absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* c
                                 const void* q, int32_t budget_tokens, void* out, void* ws,
                                 size_t ws_bytes, uint32_t flags, void* stream) {
     ABSP_TRACE("absp_decode_step_ex");
-    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX)) != 0)
+    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX |
+                                        ABSP_STEP_DIAG_WAIT_TIMEOUT)) != 0)
         return ABSP_ERR_INVALID_ARG;
     return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
                       stream, flags);
@@ -391,7 +409,8 @@ absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* 
                                  int32_t budget_tokens, int32_t* sel, int32_t* sel_count,
                                  void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
     ABSP_TRACE("absp_score_select_ex");
-    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_GROUP_MAX)) != 0) return ABSP_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<uint32_t>(ABSP_STEP_GROUP_MAX | ABSP_STEP_DIAG_WAIT_TIMEOUT)) != 0)
+        return ABSP_ERR_INVALID_ARG;
     return run_decode(kModeSelect, kv, cent, q, budget_tokens, sel, sel_count, nullptr, ws,
                       ws_bytes, stream, flags);
 }

@@ -115,20 +115,24 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) 
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after ~1 s.  On timeout
-// the error word records ABSP_ERR_TIMEOUT and the caller carries on (so that
-// every later cluster barrier is still reached); results are then garbage
-// and the host sees the error.
+// Default limit of a bounded device wait.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+// Wait for phase `parity` of an mbarrier, giving up after `limit_ns`.  On
+// timeout the error word records ABSP_ERR_TIMEOUT (detail = `where`) and the
+// caller carries on (so that every later cluster barrier is still reached);
+// results are then garbage and the host sees the error.
 template <bool CLUSTER_ACQUIRE = false>
 __device__ __forceinline__ void mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  int32_t* err, int where) {
+                                                  int32_t* err, int where,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     auto poll = [&] {
         return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
     };
     if (poll()) return;
     const uint64_t t0 = globaltimer_ns();
     while (!poll()) {
-        if (globaltimer_ns() - t0 > 1000000000ull) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             set_error(err, ABSP_ERR_TIMEOUT, where);
             return;
         }
@@ -216,6 +220,12 @@ __device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+__device__ __forceinline__ int32_t dsmem_ld_s32(uint32_t addr) {
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 // ------------------------------------------- programmatic dependent launch --
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -291,7 +301,8 @@ absp_status check_cent(const absp_centroids* c);
 // Build step (centroids.cu)
 struct BuildWs {
     int32_t* err;
-    unsigned long long* minmax;   // mins [S][Hkv][128] then maxes, order-mapped fp64
+    unsigned long long* minmax;   // mins [S][Hkv][128], then mins of the negated values
+                                  // (= -max), order-mapped fp64 keys
     double* cent;                 // [S][rows_per_seq][128]
 };
 BuildWs build_ws_layout(void* ws, const KvDesc& kv);
@@ -300,6 +311,13 @@ cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st);
 // format: ABSP_CENTROIDS_INT4 (codes + scale + zp) or ABSP_CENTROIDS_BF16
 cudaError_t launch_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
                             int32_t* zp, int format, cudaStream_t st);
+
+// Steps 1-2 in as few launches as the layer allows: one fused cluster
+// kernel when every head's centroids fit on a cluster, else build + quantize
+// (centroids.cu).  `w` is used for its error word, and fully by the
+// two-pass path.
+cudaError_t launch_build_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
+                                  int32_t* zp, int format, cudaStream_t st);
 
 // Incremental tail-row update after appended tokens (centroids.cu)
 cudaError_t launch_append(const KvDesc& kv, uint8_t* codes, const float* scale, const int32_t* zp,
@@ -323,6 +341,7 @@ struct DecodeArgs {
     int32_t nmax;                 // bound on blocks per head for this layer
     int32_t cfmt;                 // centroid format (ABSP_CENTROIDS_*)
     int32_t group_max;            // score = max over the GQA group's heads
+    int32_t diag_timeout;         // ABSP_STEP_DIAG_WAIT_TIMEOUT: the failure-path diagnostic
 };
 // early_prefetch: codes, parameters, lengths and page table are read before
 // the programmatic-dependency wait (only the query after it).

@@ -58,8 +58,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kStageRows = 256;                      // code rows per bulk stage
-constexpr int kStages = 2;                           // ring stages in region A
-constexpr int kMaxStages = 4;                        // plus up to 2 in region B's free tail
+constexpr int kStages = 2;                           // code ring stages, at least
+constexpr int kMaxStages = 4;                        // and at most
 constexpr int kStageBytes = kStageRows * kRowBytes;  // 16 KiB
 constexpr int kPageSmem = 4 * 2048;                  // K lo/hi, V lo/hi halves
 constexpr int kBins = 1024;                          // value histogram
@@ -83,18 +83,21 @@ struct Params {
     float qk_scale_log2;          // log2(e) / sqrt(128)
     uint32_t regA_off;            // byte offsets inside the aligned smem base
     uint32_t small_off;
+    uint32_t qs_off;              // the group's queries, after Small
     uint32_t scratch_off;         // select scratch inside region B
     uint32_t wg_off;              // per-head weights inside region B
     int32_t nstages;              // code ring stages (kStages .. kMaxStages)
-    uint32_t xstage_off;          // ring stages past kStages inside region B
+    uint32_t ring_off;            // code ring inside region B, past the select scratch
 };
 
 // per-head score weights for the group-max variant: [G][8 lanes][20]
 // floats (16 used), padded so the 8 lanes of a row read distinct banks
 constexpr int kWgStride = 160;
 
+constexpr int kPtStage = 512;    // page-table entries a CTA stages for its own rows
+
 struct Small {                    // fixed-size shared scratch
-    __nv_bfloat16 qs[ABSP_MAX_GROUP * kD];  // the group's queries (full mode)
+    int32_t pt[kPtStage];         // page ids of the pages of this CTA's scored rows
     unsigned long long bar_code[kMaxStages];
     unsigned long long bar_page[kWarps];
     unsigned long long bar_merge;
@@ -102,13 +105,12 @@ struct Small {                    // fixed-size shared scratch
     float2 cmm[16];               // (min, max) of each cluster CTA's scores
     int32_t misc[16];
     float red[2][kWarps];
-    float w[kD];                  // qbar[ch] * scale[ch]
+    alignas(16) float w[kD];      // qbar[ch] * scale[ch] (pre-scaled for INT4 sum scores)
+    float kz[8];                  // per lane group: sum_ch w zp, at the group's scale
+    float xs[8];                  // per lane group: 2^X
     float zb[kD];                 // 2^23 + zp[ch]
     float zf[kD];                 // zp[ch]
-    uint32_t scan[kWarps];
-    float fw[ABSP_MAX_GROUP * kWarps];  // warp merge: exp2(m_w - M) per (row, warp)
-    float rowM[ABSP_MAX_GROUP];          //   and the row's M and L
-    float rowL[ABSP_MAX_GROUP];
+    alignas(16) uint32_t scan[kWarps];
 };
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -157,34 +159,6 @@ __device__ __forceinline__ float int4_dot16(uint2 x, const float (&w)[16], float
     return a0 + a1;
 }
 
-// Softmax merge weights of n partials (m_i, l_i) per row, n a power of two
-// <= 32, for `rows` rows: partial i of row r is at [i * rows + r].  One
-// thread per (row, partial) pair, the pairs of a row on n consecutive lanes;
-// every thread of the block calls this.  Writes f[r * n + i] = exp2(m_i - M)
-// (normalised by 1 / L when `normalise`) and, when given, M and L per row,
-// with M = max_i m_i and L = sum_i l_i exp2(m_i - M); a row with no valid
-// token (M = -inf) gets zero weights.
-__device__ __forceinline__ void merge_factors(const float* m, const float* l, int rows, int n,
-                                              float* f, float* rowM, float* rowL, bool normalise) {
-    const int tid = threadIdx.x;
-    const int pairs = rows * n;
-    if (tid >= ((pairs + 31) & ~31)) return;  // whole warps only (full-mask shuffles)
-    const bool act = tid < pairs;
-    const int row = act ? tid / n : 0, i = act ? tid % n : 0;
-    const float mi = act ? m[i * rows + row] : -INFINITY;
-    float M = mi;
-    for (int o = 1; o < n; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float e = M != -INFINITY ? exp2f(mi - M) : 0.0f;
-    float L = act ? l[i * rows + row] * e : 0.0f;
-    for (int o = 1; o < n; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (!act) return;
-    f[row * n + i] = normalise ? (L > 0.0f ? e * (1.0f / L) : 0.0f) : e;
-    if (rowM != nullptr && i == 0) {
-        rowM[row] = M;
-        rowL[row] = L;
-    }
-}
-
 // Sums of four rows' partial dot products over the 8 lanes of a group
 // (lanes 8g .. 8g + 7), returned to every lane of the group.  A transpose
 // reduction: each butterfly step halves the rows a lane carries, so lane
@@ -222,18 +196,6 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* scan) 
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) base += w < warp ? t[w] : 0u;
     return base + inc - v;
-}
-
-// Warp-wide exclusive prefix sum.
-__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v) {
-    const int lane = threadIdx.x & 31;
-    uint32_t inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += t;
-    }
-    return inc - v;
 }
 
 // Threshold of the top-k by 4 passes of 8-bit radix select over the
@@ -312,32 +274,24 @@ __device__ __noinline__ void compact_by_threshold(const float* sc, int n, uint32
 }
 
 // Entries [lo, hi) of the ascending list of the set bits of
-// bitmap[0..nwords), by one warp: out[pos - lo] = bit index.
-__device__ __forceinline__ void warp_extract_bitmap(const uint32_t* bitmap, int nwords,
-                                                    int32_t* out, int lo, int hi) {
-    // run once per CTA by one warp: compact loops rather than unrolled ones
-    // keep this cold code small
-    const int lane = threadIdx.x & 31;
-    const int wpl = (nwords + 31) / 32;
-    const int j0 = min(nwords, lane * wpl), j1 = min(nwords, j0 + wpl);
-    uint32_t cnt = 0;
-#pragma unroll 1
-    for (int j = j0; j < j1; ++j) cnt += __popc(bitmap[j]);
-    int pos = static_cast<int>(warp_excl_scan(cnt));
-    if (pos + static_cast<int>(cnt) <= lo || pos >= hi) return;
-#pragma unroll 1
-    for (int j = j0; j < j1 && pos < hi; ++j) {
-        uint32_t bits = bitmap[j];
-        const int c = __popc(bits);
-        if (pos + c <= lo) {  // the whole word lies before the wanted entries
-            pos += c;
-            continue;
-        }
-        while (bits && pos < hi) {
-            if (pos >= lo) out[pos - lo] = j * 32 + (__ffs(bits) - 1);
-            ++pos;
-            bits &= bits - 1u;
-        }
+// bitmap[0..nwords), by the whole block: warp w owns the contiguous words
+// [w * wpw, (w + 1) * wpw) and wcnt[w] holds the number of set bits in them.
+// Each lane places its own bit of every word: position = the set bits of the
+// warps before, of the words before in its run, and of the lanes below.
+__device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int nwords, int wpw,
+                                                     const uint32_t* wcnt, int32_t* out, int lo,
+                                                     int hi) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t pos = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) pos += w < warp ? wcnt[w] : 0u;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int j0 = min(nwords, warp * wpw), j1 = min(nwords, j0 + wpw);
+    for (int j = j0; j < j1 && static_cast<int>(pos) < hi; ++j) {
+        const uint32_t bits = bitmap[j];
+        const int at = static_cast<int>(pos + __popc(bits & lt));
+        if (((bits >> lane) & 1u) && at >= lo && at < hi) out[at - lo] = j * 32 + lane;
+        pos += __popc(bits);
     }
 }
 
@@ -345,9 +299,10 @@ __device__ __forceinline__ void warp_extract_bitmap(const uint32_t* bitmap, int 
 // index order; only list entries [lo, hi) are written, to out[0 .. hi-lo).
 // [mn, mx] is the range of the scores.  The kBins histogram bins at the
 // start of `scratch` must be zero on entry.  n <= 65535.
+template <typename OnBoundary>
 __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float mn, float mx,
                                            int32_t* out, int lo, int hi, uint32_t* scratch,
-                                           Small& sm) {
+                                           Small& sm, OnBoundary&& on_boundary) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (k >= n) {
         for (int i = max(0, lo) + tid; i < min(n, hi); i += kThreads) out[i - lo] = i;
@@ -364,16 +319,37 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
         return;
     }
     if (inv < INFINITY) {
-        // histogram of the scores over kBins equal bins of [mn, mx]; the
-        // bins were zeroed by the caller
-        constexpr int U = 8;
-        for (int b = tid; b < n; b += kThreads * U) {
-            float x[U];
+        // histogram of the scores over kBins equal bins of [mn, mx] (the
+        // bins were zeroed by the caller).  Warp w owns the ballot words
+        // [w * wpw, (w + 1) * wpw) (32 scores each) here and in the ballot
+        // pass below; the bins of a thread's first 8 words stay in
+        // registers for that pass.
+        const int nwords = (n + 31) / 32;
+        const int wpw = (nwords + kWarps - 1) / kWarps;
+        const int j0 = min(nwords, warp * wpw), j1 = min(nwords, j0 + wpw);
+        constexpr int V = 8;
+        int kbin[V];
+        float kx[V];
+        for (int jb = j0; jb < j1; jb += V) {
+            float x[V];
+            int bn[V];
 #pragma unroll
-            for (int u = 0; u < U; ++u) x[u] = b + u * kThreads < n ? sc[b + u * kThreads] : mn;
+            for (int v = 0; v < V; ++v) {
+                const int i = (jb + v) * 32 + lane;
+                const bool live = jb + v < j1 && i < n;
+                x[v] = live ? sc[i] : mn;
+                bn[v] = live ? value_bin(x[v], mn, inv) : -1;
+            }
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (b + u * kThreads < n) atomicAdd(&hist[value_bin(x[u], mn, inv)], 1u);
+            for (int v = 0; v < V; ++v)
+                if (bn[v] >= 0) atomicAdd(&hist[bn[v]], 1u);
+            if (jb == j0) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    kbin[v] = bn[v];
+                    kx[v] = x[v];
+                }
+            }
         }
         __syncthreads();
         {
@@ -399,29 +375,35 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
         }
         __syncthreads();
         const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
+        on_boundary(bstar, mn, inv);
         if (m <= kMaxCand) {
             // one pass: a ballot word per 32 scores marks those above bin
             // bstar (selected); the scores inside bstar become candidates,
-            // all of them selected when the whole bin is needed
+            // all of them selected when the whole bin is needed.  Warp w
+            // owns the contiguous words [w * wpw, (w + 1) * wpw) and counts
+            // their selected scores.
             const bool all_in = need == m;
-            const int nwords = (n + 31) / 32;
-            constexpr int V = 8;
-            for (int w0 = warp; w0 < nwords; w0 += kWarps * V) {
+            uint32_t cnt = 0;
+            for (int jb = j0; jb < j1; jb += V) {
                 float x[V];
+                int bnv[V];
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    const int i = (w0 + v * kWarps) * 32 + lane;
-                    x[v] = (w0 + v * kWarps < nwords && i < n) ? sc[i] : mn;
+                    const int i = (jb + v) * 32 + lane;
+                    const bool live = jb + v < j1 && i < n;
+                    x[v] = jb == j0 ? kx[v] : (live ? sc[i] : mn);
+                    bnv[v] = jb == j0 ? kbin[v] : (live ? value_bin(x[v], mn, inv) : -1);
                 }
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    const int wd = w0 + v * kWarps;
+                    const int wd = jb + v;
                     const int i = wd * 32 + lane;
-                    const bool live = wd < nwords && i < n;
-                    const int bn = value_bin(x[v], mn, inv);
+                    const bool live = wd < j1 && i < n;
+                    const int bn = bnv[v];
                     const uint32_t gw =
                         __ballot_sync(0xffffffffu, live && (bn > bstar || (all_in && bn == bstar)));
-                    if (lane == 0 && wd < nwords) inw[wd] = gw;
+                    if (lane == 0 && wd < j1) inw[wd] = gw;
+                    cnt += __popc(gw);
                     if (!all_in && live && bn == bstar) {
                         const int pos = atomicAdd(&sm.misc[3], 1);
                         ckey[pos] = order_key(x[v]);
@@ -429,23 +411,44 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                     }
                 }
             }
+            if (lane == 0) sm.scan[warp] = cnt;
             __syncthreads();
             if (!all_in) {
                 // exact rank among the candidates: larger key first, ties to
                 // the lower index; the `need` best join the selection
-                for (int c = tid; c < m; c += kThreads) {
-                    const uint32_t key = ckey[c];
-                    const int idx = cidx[c];
-                    int rank = 0;
-                    for (int j = 0; j < m; ++j) {
-                        const uint32_t kj = ckey[j];
-                        rank += (kj > key) || (kj == key && cidx[j] < idx);
+                if (m <= 32) {
+                    if (warp == 0) {
+                        const uint32_t key = lane < m ? ckey[lane] : 0u;
+                        const int idx = lane < m ? cidx[lane] : 0x7fffffff;
+                        int rank = 0;
+                        for (int j = 0; j < m; ++j) {
+                            const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+                            const int ij = __shfl_sync(0xffffffffu, idx, j);
+                            rank += (kj > key) || (kj == key && ij < idx);
+                        }
+                        if (lane < m && rank < need) {
+                            atomicOr(&inw[idx >> 5], 1u << (idx & 31));
+                            atomicAdd(&sm.scan[(idx >> 5) / wpw], 1u);
+                        }
                     }
-                    if (rank < need) atomicOr(&inw[idx >> 5], 1u << (idx & 31));
+                } else {
+                    for (int c = tid; c < m; c += kThreads) {
+                        const uint32_t key = ckey[c];
+                        const int idx = cidx[c];
+                        int rank = 0;
+                        for (int j = 0; j < m; ++j) {
+                            const uint32_t kj = ckey[j];
+                            rank += (kj > key) || (kj == key && cidx[j] < idx);
+                        }
+                        if (rank < need) {
+                            atomicOr(&inw[idx >> 5], 1u << (idx & 31));
+                            atomicAdd(&sm.scan[(idx >> 5) / wpw], 1u);
+                        }
+                    }
                 }
                 __syncthreads();
             }
-            if (warp == 0) warp_extract_bitmap(inw, nwords, out, lo, hi);
+            block_extract_bitmap(inw, nwords, wpw, sm.scan, out, lo, hi);
             __syncthreads();
             return;
         }
@@ -461,7 +464,11 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 #define ABSP_DECODE_MIN_BLOCKS 2  // CTAs per SM the register budget is built for
 #endif
 
-template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM>
+// DIAG: the failure-path diagnostic (ABSP_STEP_DIAG_WAIT_TIMEOUT): the
+// score barrier expects 16 bytes that are never sent and every bounded wait
+// gives up after 1 ms, so the score wait runs out, records ABSP_ERR_TIMEOUT
+// and the kernel carries on to its normal end.
+template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM, bool DIAG>
 __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
@@ -469,15 +476,19 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     // 1024-byte aligned base, derived from the shared array by a byte offset
     // so that every access below stays in the shared address space
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* regB = base;                        // scores / pages / warp merge
-    uint8_t* regA = base + p.regA_off;           // code ring / cluster merge
+    uint8_t* regB = base;                        // scores + ring / pages / warp merge
+    uint8_t* regA = base + p.regA_off;           // cluster merge receive buffers
     Small& sm = *reinterpret_cast<Small*>(base + p.small_off);
-    int32_t* sel_s = reinterpret_cast<int32_t*>(base + p.small_off + sizeof(Small));
+    __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(base + p.qs_off);  // [G][128]
+    int32_t* sel_s = reinterpret_cast<int32_t*>(base + p.qs_off + p.kv.G * kD * 2);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t C = cluster_nctarank();
     const uint32_t rank = cluster_ctarank();
-    const int pair = blockIdx.x / C;
+    // C (a power of two), bs and bs / 16 are powers of two: shifts, not
+    // divisions, on the dependent path
+    const int lgC = __ffs(static_cast<int>(C)) - 1;
+    const int pair = blockIdx.x >> lgC;
     const int Hkv = p.kv.Hkv, G = p.kv.G;
     const int s = pair / Hkv, h = pair % Hkv;
     const int bs = p.kv.bs[h];
@@ -488,12 +499,13 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     // centroid rows: 64 B of INT4 codes, or 256 B of bf16 centroids
     constexpr int kRow = BF16C ? 2 * kD : kRowBytes;
     constexpr int kSRows = kStageBytes / kRow;         // rows per bulk stage
+    constexpr uint64_t kWaitNs = DIAG ? 1000000ull : kWaitLimitNs;
 
     if (tid == 0) {
         for (int i = 0; i < kMaxStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
         for (int w = 0; w < kWarps; ++w) mbar_init(smem_u32(&sm.bar_page[w]), 1);
         mbar_init(smem_u32(&sm.bar_score), 1);
-        if (C > 1) mbar_init(smem_u32(&sm.bar_merge), C - 1);
+        mbar_init(smem_u32(&sm.bar_merge), 1);
         fence_mbar_init();
     }
     // Without EARLY nothing in global memory is read before this wait.
@@ -506,27 +518,48 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         if (tid == 0 && rank == 0 && h == 0) set_error(p.err, ABSP_ERR_DEVICE_FAULT, s);
         len = 0;
     }
-    const int n = (len + bs - 1) / bs;
+    const int lgbs = __ffs(bs) - 1, lgspb = lgbs - 4;
+    const int n = (len + bs - 1) >> lgbs;
     // rows of this CTA: a contiguous range, a multiple of 4 rows long
-    const int per = ((n + static_cast<int>(C) - 1) / static_cast<int>(C) + 3) & ~3;
+    const int per = (((n + static_cast<int>(C) - 1) >> lgC) + 3) & ~3;
     const int r0 = min(n, static_cast<int>(rank) * per);
     const int nrows = min(n, r0 + per) - r0;
     const int nchunks = (nrows + kSRows - 1) / kSRows;
+    const int npg = (len + kPage - 1) / kPage;
+    // The selected blocks' page ids: in the fused mode each CTA stages the
+    // page-table entries of its own scored rows in shared memory and the
+    // attending CTAs read them through distributed shared memory, when the
+    // slice fits and every warp attends at most 32 pages (all lookups then
+    // happen once, at the start of the attention, while every CTA of the
+    // cluster is still running: none leaves before it received every other
+    // CTA's merge partial).  Uniform over a cluster.
+    const int Ksel = min(n, max(1, p.budget >> lgbs));
+    const bool stage_pt = kSelect && kAttend && per > 0 && per * spb <= kPtStage &&
+                          ((Ksel * spb + static_cast<int>(C) - 1) >> lgC) <= 32 * kWarps;
+    int ptv[kPtStage / kThreads];
+#pragma unroll
+    for (int u = 0; u < kPtStage / kThreads; ++u) {
+        const int i = tid + u * kThreads;
+        const int lp = r0 * spb + i;
+        ptv[u] = stage_pt && i < nrows * spb && lp < npg ? pt[lp] : -1;
+    }
     const uint8_t* cbase =
         p.codes + (static_cast<int64_t>(s) * p.kv.rows_per_seq + p.kv.row_base[h] + r0) * kRow;
-    // code ring: stages 0, 1 in region A, further ones in region B past the
-    // scores and select scratch (free until the attention phase)
+    // code ring: region B past the scores and select scratch (region B is
+    // free for it until the attention phase)
     const int NS = p.nstages;
-    auto stage_buf = [&](int st) -> uint8_t* {
-        return st < kStages ? regA + st * kStageBytes
-                            : regB + p.xstage_off + (st - kStages) * kStageBytes;
-    };
+    auto stage_buf = [&](int st) -> uint8_t* { return regB + p.ring_off + st * kStageBytes; };
     if (tid == 0) {
+        if (kAttend && C > 1)
+            // every other CTA's slice of its partial: G rows x 128/C
+            // channels, and (M, L) per row
+            mbar_arrive_expect_tx(smem_u32(&sm.bar_merge),
+                                  (C - 1) * (G * (kD / C) * 4 + 8 * G));
         if (kSelect && (MODE != kModeSelect || rank == 0))
             // every CTA's scores but this one's own (plain stores), and
             // every CTA's (min, max)
             mbar_arrive_expect_tx(smem_u32(&sm.bar_score),
-                                  16 * ((n + 3) / 4 - (nrows + 3) / 4) + 8 * C);
+                                  16 * ((n + 3) / 4 - (nrows + 3) / 4) + 8 * C + (DIAG ? 16 : 0));
         if (kSelect) {
             for (int c = 0; c < min(nchunks, NS); ++c) {
                 const int rows = min(kSRows, nrows - c * kSRows);
@@ -543,9 +576,8 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     // B0 arrive (release: the barrier set-up above is visible cluster-wide
     // once B0 completes); matched by the wait before the first remote access.
     cluster_arrive();
-    if constexpr (kAttend) {
+    if (kAttend && !stage_pt) {
         // the attention phase reads page-table entries of this sequence
-        const int npg = (len + kPage - 1) / kPage;
         for (int i = tid * 32; i < npg; i += kThreads * 32) prefetch_l2(pt + i);
     }
     float scl = 0.0f;
@@ -570,7 +602,11 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
 
     if constexpr (kSelect) {
         // ---------------------------------------------------- A: score --
-        K = min(n, max(1, p.budget / bs));
+        K = Ksel;
+        if (stage_pt) {
+#pragma unroll
+            for (int u = 0; u < kPtStage / kThreads; ++u) sm.pt[tid + u * kThreads] = ptv[u];
+        }
         if (tid < kD) {
             const __nv_bfloat16* qh = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD + tid;
             // the group's queries are read once (they may live in host
@@ -578,17 +614,40 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             float qb = 0.0f;
             for (int j = 0; j < G; ++j) {
                 const __nv_bfloat16 qv = qh[j * kD];
-                sm.qs[j * kD + tid] = qv;
+                qs[j * kD + tid] = qv;
                 qb += __bfloat162float(qv);
             }
-            sm.w[tid] = BF16C ? qb : qb * scl;
+            const float wv = BF16C ? qb : qb * scl;
+            sm.w[tid] = wv;
             sm.zb[tid] = 8388608.0f + static_cast<float>(zpv);
             sm.zf[tid] = static_cast<float>(zpv);
+            if constexpr (!BF16C && !GM) {
+                // INT4 sum scores: sum_ch w (code - zp) = sum_ch w code -
+                // sum_ch w zp.  Lane group `sub` (channels 16 sub .. 16 sub
+                // + 15, the 16 threads tid & ~15 here) works at scale 2^-X,
+                // X from its largest |w| (2^e <= max|w| < 2^(e+1)): the
+                // pre-scaled weights w 2^(149 - 4j - X) stay below 2^126 and
+                // products of the larger weights are normal.  Each thread
+                // prepares its channel once for the 32 lanes that use it.
+                float mw = fabsf(wv), zs = wv * static_cast<float>(zpv);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) {
+                    mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+                    zs += __shfl_xor_sync(0xffffffffu, zs, o);
+                }
+                const int e = static_cast<int>((__float_as_uint(mw) >> 23) & 0xFFu) - 127;
+                const int X = min(126, max(22, 24 + e));
+                sm.w[tid] = wv * __uint_as_float(static_cast<uint32_t>(276 - X - 4 * (tid & 3)) << 23);
+                if ((tid & 15) == 0) {
+                    sm.kz[tid >> 4] = zs * __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
+                    sm.xs[tid >> 4] = __uint_as_float(static_cast<uint32_t>(127 + X) << 23);
+                }
+            }
             if constexpr (GM) {
                 float* wg = reinterpret_cast<float*>(regB + p.wg_off);
                 const int slot = (tid >> 4) * 20 + (tid & 15);
                 for (int j = 0; j < G; ++j) {
-                    const float qj = __bfloat162float(sm.qs[j * kD + tid]);
+                    const float qj = __bfloat162float(qs[j * kD + tid]);
                     wg[j * kWgStride + slot] = BF16C ? qj : qj * scl;
                 }
             }
@@ -599,28 +658,20 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         float kz = 0.0f;  // this lane's share of sum_ch w[ch] * zp[ch], scaled
         float xs = 1.0f;  // 2^X: undoes the lane's scale on its partial sum
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            wr[k] = sm.w[sub * 16 + k];
-            zr[k] = sm.zb[sub * 16 + k];
+        for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 v = *reinterpret_cast<const float4*>(&sm.w[sub * 16 + 4 * k4]);
+            wr[4 * k4] = v.x;
+            wr[4 * k4 + 1] = v.y;
+            wr[4 * k4 + 2] = v.z;
+            wr[4 * k4 + 3] = v.w;
+        }
+        if constexpr (GM) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) zr[k] = sm.zb[sub * 16 + k];
         }
         if constexpr (!BF16C && !GM) {
-            // INT4 sum scores: sum_ch w (code - zp) = sum_ch w code - sum_ch w zp.
-            // The lane works at scale 2^-X, X from its largest |w| (2^e <=
-            // max|w| < 2^(e+1)): the pre-scaled weights w 2^(149 - 4j - X)
-            // stay below 2^126 and products of the larger weights are normal.
-            float mw = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                kz = fmaf(wr[k], sm.zf[sub * 16 + k], kz);
-                mw = fmaxf(mw, fabsf(wr[k]));
-            }
-            const int e = static_cast<int>((__float_as_uint(mw) >> 23) & 0xFFu) - 127;
-            const int X = min(126, max(22, 24 + e));
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                wr[k] *= __uint_as_float(static_cast<uint32_t>(276 - X - 4 * (k & 3)) << 23);
-            kz *= __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
-            xs = __uint_as_float(static_cast<uint32_t>(127 + X) << 23);
+            kz = sm.kz[sub];
+            xs = sm.xs[sub];
         }
         float* scores = reinterpret_cast<float*>(regB);
         const uint32_t scores_u32 = smem_u32(scores);
@@ -635,11 +686,13 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         // 8-lane group's scores of rows r4 .. r4 + 3 of a stage (values for
         // rows past `rows` are discarded here).
         auto chunk_loop = [&](auto&& score4) {
+#pragma unroll 1
             for (int c = 0; c < nchunks; ++c) {
                 const int stage = c % NS;
-                mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / NS) & 1, p.err, 1);
+                mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / NS) & 1, p.err, 1, kWaitNs);
                 const int rows = min(kSRows, nrows - c * kSRows);
                 const uint8_t* sbuf = stage_buf(stage);
+#pragma unroll 1
                 for (int rb = 0; rb < rows; rb += 4 * (kThreads / 8)) {
                     const int r4 = rb + 4 * grp;
                     const float4 q = score4(sbuf, r4, rows);
@@ -800,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         // select-only: CTA 0 alone receives and selects
         if (MODE == kModeSelect && rank != 0) return;
         // ------------------------------------- B: every score arrived --
-        mbar_wait_bounded<true>(bar_score, 0, p.err, 4);
+        mbar_wait_bounded<true>(bar_score, 0, p.err, 4, kWaitNs);
 
         // --------------------------------------------------- C: select --
         float smin = INFINITY, smax = -INFINITY;
@@ -818,13 +871,32 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             // this CTA attends list entries [sel_lo, sel_hi): the blocks of
             // its share [pb, pe) of the K * bs/16 selected pages
             const int P = K * spb;
-            const int pb = static_cast<int>(static_cast<uint32_t>(P) * rank / C);  // P*C < 2^21
-            const int pe = static_cast<int>(static_cast<uint32_t>(P) * (rank + 1) / C);
-            sel_lo = pb / spb;
-            sel_hi = pe > pb ? (pe - 1) / spb + 1 : sel_lo;
+            const int pb = static_cast<int>((static_cast<uint32_t>(P) * rank) >> lgC);  // P*C < 2^21
+            const int pe = static_cast<int>((static_cast<uint32_t>(P) * (rank + 1)) >> lgC);
+            sel_lo = pb >> lgspb;
+            sel_hi = pe > pb ? ((pe - 1) >> lgspb) + 1 : sel_lo;
         }
+        // once the boundary bin is known, the pages of this CTA's own rows
+        // that score above it (selected whatever the boundary ranking gives)
+        // start their way into L2 while the selection is finished
+        auto prefetch_sure = [&](int bstar, float mn, float inv) {
+            if constexpr (kAttend) {
+                if (!stage_pt) return;
+                for (int r = tid; r < nrows; r += kThreads) {
+                    if (value_bin(scores[r0 + r], mn, inv) <= bstar) continue;
+                    for (int jj = 0; jj < spb; ++jj) {
+                        const int lp = (r0 + r) * spb + jj;
+                        const int phys = sm.pt[r * spb + jj];
+                        if (lp >= npg || phys < 0 || phys >= p.kv.num_phys_pages) break;
+                        const int64_t off = (static_cast<int64_t>(phys) * Hkv + h) * (kPage * kD);
+                        bulk_prefetch_l2(p.kv.k_pages + off, kPage * kD * 2);
+                        bulk_prefetch_l2(p.kv.v_pages + off, kPage * kD * 2);
+                    }
+                }
+            }
+        };
         block_topk(scores, n, K, smin, smax, sel_s, sel_lo, sel_hi,
-                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm);
+                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm, prefetch_sure);
         if (MODE == kModeSelect) {
             int32_t* dst = p.sel + (static_cast<int64_t>(s) * Hkv + h) * p.kmax;
             for (int i = tid; i < K; i += kThreads) dst[i] = sel_s[i];  // [0, K) held
@@ -853,8 +925,8 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     if constexpr ((MODE & kModeAttend) != 0) {
         // --------------------------------------------------- D: attend --
         const int P = K * spb;
-        const int pb = static_cast<int>(static_cast<uint32_t>(P) * rank / C);  // P*C < 2^21
-        const int pe = static_cast<int>(static_cast<uint32_t>(P) * (rank + 1) / C);
+        const int pb = static_cast<int>((static_cast<uint32_t>(P) * rank) >> lgC);  // P*C < 2^21
+        const int pe = static_cast<int>((static_cast<uint32_t>(P) * (rank + 1)) >> lgC);
         const int cnt_w = pe - pb > warp ? (pe - pb - warp + kWarps - 1) / kWarps : 0;
         const int g = lane >> 2, t4 = lane & 3;
         // queries: the copy made while scoring; attend-only launches make it
@@ -863,10 +935,10 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             const uint32_t* qsrc = reinterpret_cast<const uint32_t*>(
                 p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD);
             for (int i = tid; i < G * kD / 2; i += kThreads)
-                reinterpret_cast<uint32_t*>(sm.qs)[i] = qsrc[i];
+                reinterpret_cast<uint32_t*>(qs)[i] = qsrc[i];
             __syncthreads();
         }
-        const __nv_bfloat16* qg = sm.qs;
+        const __nv_bfloat16* qg = qs;
         float o[16][4];
 #pragma unroll
         for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
@@ -875,26 +947,53 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         const float qks = p.qk_scale_log2;
         uint8_t* wbuf = regB + warp * kPageSmem;  // this warp's page buffer
 
-        // page i of this warp: selection entry, bounds checks, tensor copies
+        // Pages of this warp, 32 at a time: lane l resolves page c0 + l into
+        // its physical page id and valid token count (one parallel round of
+        // page-table reads instead of one read per page); a page that is
+        // past the sequence end, or whose id is out of range, gets 0 tokens.
+        int my_phys = 0, my_valid = 0, c0 = 0;
+        auto resolve = [&](int i0) {
+            c0 = i0;
+            my_phys = 0;
+            my_valid = 0;
+            const int i = i0 + lane;
+            if (i >= cnt_w) return;
+            const int j = pb + warp + kWarps * i;
+            const int b = sel_s[(j >> lgspb) - sel_lo];
+            if (b < 0) return;
+            const int lp = b * spb + (j & (spb - 1));
+            const int valid = min(kPage, len - lp * kPage);
+            if (valid <= 0) return;
+            int phys;
+            if (stage_pt) {
+                // staged by the CTA that scored block b
+                // b / per by a float reciprocal, corrected to the exact
+                // quotient (b < 2^14, per >= 4)
+                int owner = __float2int_rz((static_cast<float>(b) + 0.5f) *
+                                           __frcp_rn(static_cast<float>(per)));
+                owner += (owner + 1) * per <= b;
+                owner -= owner * per > b;
+                int32_t* e = &sm.pt[lp - owner * per * spb];
+                phys = owner == static_cast<int>(rank) ? *e
+                                                        : dsmem_ld_s32(dsmem_addr(smem_u32(e), owner));
+            } else {
+                phys = pt[lp];
+            }
+            if (phys < 0 || phys >= p.kv.num_phys_pages) {
+                set_error(p.err, ABSP_ERR_DEVICE_FAULT, s);
+                return;
+            }
+            my_phys = phys;
+            my_valid = valid;
+        };
+
+        // page i of this warp: tensor copies of its K and V slices (every
+        // lane calls this; lane 0 issues)
         auto issue = [&](int i) -> int {
-            int valid = 0;
+            if (i >= c0 + 32) resolve(i);
+            const int valid = __shfl_sync(0xffffffffu, my_valid, i & 31);
+            const int phys = __shfl_sync(0xffffffffu, my_phys, i & 31);
             if (lane == 0) {
-                const int j = pb + warp + kWarps * i;
-                const int b = sel_s[j / spb - sel_lo];
-                int phys = -1;
-                if (b >= 0) {
-                    const int lp = b * spb + (j % spb);
-                    valid = min(kPage, len - lp * kPage);
-                    if (valid > 0) {
-                        phys = pt[lp];
-                        if (phys < 0 || phys >= p.kv.num_phys_pages) {
-                            set_error(p.err, ABSP_ERR_DEVICE_FAULT, s);
-                            valid = 0;
-                        }
-                    } else {
-                        valid = 0;
-                    }
-                }
                 const uint32_t bar = smem_u32(&sm.bar_page[warp]);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, valid > 0 ? kPageSmem : 0);
@@ -907,31 +1006,30 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                     tma_load_2d(dst + 6144, &tmv, 64, y, bar);
                 }
             }
-            return __shfl_sync(0xffffffffu, valid, 0);
+            return valid;
         };
 
-        // page i of this warp: its K and V slices into L2, ahead of the copy
+        // page i of this warp into L2 ahead of its copy, when it is among
+        // the pages resolved (every lane calls this; lane 0 issues)
         auto prefetch = [&](int i) {
-            if (lane != 0 || i >= cnt_w) return;
-            const int j = pb + warp + kWarps * i;
-            const int b = sel_s[j / spb - sel_lo];
-            if (b < 0) return;
-            const int lp = b * spb + (j % spb);
-            if (lp * kPage >= len) return;
-            const int phys = pt[lp];
-            if (phys < 0 || phys >= p.kv.num_phys_pages) return;
+            if (i >= cnt_w || i < c0 || i >= c0 + 32) return;
+            const int valid = __shfl_sync(0xffffffffu, my_valid, i & 31);
+            const int phys = __shfl_sync(0xffffffffu, my_phys, i & 31);
+            if (lane != 0 || valid <= 0) return;
             const int64_t off = (static_cast<int64_t>(phys) * Hkv + h) * (kPage * kD);
             bulk_prefetch_l2(p.kv.k_pages + off, kPage * kD * 2);
             bulk_prefetch_l2(p.kv.v_pages + off, kPage * kD * 2);
         };
 
         __syncthreads();  // every thread is done with the scores in region B
+        resolve(0);
         int vnext = cnt_w > 0 ? issue(0) : 0;
 #pragma unroll 1
         for (int i = 1; i <= ABSP_PAGE_PREFETCH; ++i) prefetch(i);
+#pragma unroll 1
         for (int i = 0; i < cnt_w; ++i) {
             const int valid = vnext;
-            mbar_wait_bounded(smem_u32(&sm.bar_page[warp]), i & 1, p.err, 2);
+            mbar_wait_bounded(smem_u32(&sm.bar_page[warp]), i & 1, p.err, 2, kWaitNs);
             if (valid > 0) {
                 uint8_t* pg = wbuf;
                 const uint32_t kb = smem_u32(pg), vb = kb + 4096;
@@ -1051,16 +1149,20 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         }
 
         // ------------------------------------------- E: merge partials --
+        // Warps merge in shared memory into this CTA's partial (O, M, L);
+        // with C > 1 CTA r owns output channels [r * 128/C, (r + 1) * 128/C)
+        // of every row, receives that slice of every CTA's partial (16-byte
+        // asynchronous stores counted on its mbarrier, its own by plain
+        // stores), merges the C partials and writes the slice.
         __syncthreads();                                   // page buffers are dead
         float* Ow = reinterpret_cast<float*>(regB);        // [warps][G][128]
         float* mw = Ow + kWarps * G * kD;                  // [warps][G]
         float* lw = mw + kWarps * G;
         if (g < G) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                Ow[(warp * G + g) * kD + t * 8 + 2 * t4] = o[t][0];
-                Ow[(warp * G + g) * kD + t * 8 + 2 * t4 + 1] = o[t][1];
-            }
+            for (int t = 0; t < 16; ++t)
+                *reinterpret_cast<float2*>(&Ow[(warp * G + g) * kD + t * 8 + 2 * t4]) =
+                    make_float2(o[t][0], o[t][1]);
             if (t4 == 0) {
                 mw[warp * G + g] = m0;
                 lw[warp * G + g] = l0;
@@ -1069,10 +1171,9 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         if constexpr (BIG_GROUP) {
             if (g + 8 < G) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    Ow[(warp * G + g + 8) * kD + t * 8 + 2 * t4] = o[t][2];
-                    Ow[(warp * G + g + 8) * kD + t * 8 + 2 * t4 + 1] = o[t][3];
-                }
+                for (int t = 0; t < 16; ++t)
+                    *reinterpret_cast<float2*>(&Ow[(warp * G + g + 8) * kD + t * 8 + 2 * t4]) =
+                        make_float2(o[t][2], o[t][3]);
                 if (t4 == 0) {
                     mw[warp * G + g + 8] = m8;
                     lw[warp * G + g + 8] = l8;
@@ -1080,69 +1181,105 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             }
         }
         __syncthreads();
-        // per (row, warp) weight exp2(m_w - M) and the row's M and L: one
-        // thread per pair, reduced over the warp's 8-lane segment
-        merge_factors(mw, lw, G, kWarps, sm.fw, sm.rowM, sm.rowL, false);
-        __syncthreads();
         if constexpr ((MODE & kModeSelect) == 0) cluster_wait();  // B0
-        float* partO = reinterpret_cast<float*>(regA);    // [C][G][128]
-        float* partM = partO + C * G * kD;                 // [C][G]
-        float* partL = partM + C * G;
         __nv_bfloat16* outp = p.out + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
-        for (int idx = tid; idx < G * kD; idx += kThreads) {
-            const int row = idx >> 7, d = idx & (kD - 1);
-            const float M = sm.rowM[row], L = sm.rowL[row];
-            float oa = 0.0f, ob = 0.0f;
+        // this CTA's partial of 4 channels of one row, with the row's M and
+        // L: the weights exp2(m_w - M) of the warp partials are computed in
+        // place by every thread of the row (a row with no valid token has
+        // M = -inf and gets zero weights)
+        auto cta_partial = [&](int row, int d, float& M, float& L) -> float4 {
+            float mv[kWarps];
+            M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kWarps; w += 2) {
-                oa = fmaf(Ow[(w * G + row) * kD + d], sm.fw[row * kWarps + w], oa);
-                ob = fmaf(Ow[((w + 1) * G + row) * kD + d], sm.fw[row * kWarps + w + 1], ob);
+            for (int w = 0; w < kWarps; ++w) {
+                mv[w] = mw[w * G + row];
+                M = fmaxf(M, mv[w]);
             }
-            const float Oacc = oa + ob;
-            if (C == 1) {
-                outp[row * kD + d] = __float2bfloat16_rn(L > 0.0f ? Oacc / L : 0.0f);
-            } else if (rank == 0) {
-                partO[row * kD + d] = Oacc;
-                if (d == 0) {
-                    partM[row] = M;
-                    partL[row] = L;
-                }
-            } else {
-                const uint32_t lo = smem_u32(&partO[(rank * G + row) * kD + d]);
-                dsmem_st_f32(dsmem_addr(lo, 0), Oacc);
-                if (d == 0) {
-                    dsmem_st_f32(dsmem_addr(smem_u32(&partM[rank * G + row]), 0), M);
-                    dsmem_st_f32(dsmem_addr(smem_u32(&partL[rank * G + row]), 0), L);
+            L = 0.0f;
+            float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const float e = M != -INFINITY ? exp2f(mv[w] - M) : 0.0f;
+                L = fmaf(lw[w * G + row], e, L);
+                const float4 v = *reinterpret_cast<const float4*>(&Ow[(w * G + row) * kD + d]);
+                a.x = fmaf(v.x, e, a.x);
+                a.y = fmaf(v.y, e, a.y);
+                a.z = fmaf(v.z, e, a.z);
+                a.w = fmaf(v.w, e, a.w);
+            }
+            return a;
+        };
+        if (C == 1) {
+#pragma unroll 1
+            for (int idx = tid; idx < G * (kD / 4); idx += kThreads) {
+                const int row = idx / (kD / 4), d = (idx % (kD / 4)) * 4;
+                float M, L;
+                const float4 a = cta_partial(row, d, M, L);
+                const float r = L > 0.0f ? 1.0f / L : 0.0f;
+                // 4-byte stores: the output is only 4-byte aligned
+                uint32_t* o2 = reinterpret_cast<uint32_t*>(outp + row * kD + d);
+                o2[0] = pack_bf16x2(a.x * r, a.y * r);
+                o2[1] = pack_bf16x2(a.z * r, a.w * r);
+            }
+            return;
+        }
+        const int ds = kD >> lgC;                           // channels per slice, >= 8
+        const int lgds = 7 - lgC;
+        float* recvO = reinterpret_cast<float*>(regA);      // [C][G][ds]
+        float* recvML = recvO + C * G * ds;                 // [C][G][2]: (M, L)
+        const uint32_t bar_merge = smem_u32(&sm.bar_merge);
+#pragma unroll 1
+        for (int idx = tid; idx < G * (kD / 4); idx += kThreads) {
+            const int row = idx / (kD / 4), d4 = idx % (kD / 4), d = d4 * 4;
+            float M, L;
+            const float4 a = cta_partial(row, d, M, L);
+            const uint32_t owner = static_cast<uint32_t>(d >> lgds);
+            float* dst = &recvO[(rank * G + row) * ds + (d - static_cast<int>(owner) * ds)];
+            if (owner == rank)
+                *reinterpret_cast<float4*>(dst) = a;
+            else
+                st_async_v4(dsmem_addr(smem_u32(dst), owner), a.x, a.y, a.z, a.w,
+                            dsmem_addr(bar_merge, owner));
+            if (d4 < static_cast<int>(C)) {   // the row's (M, L) to owner d4
+                const uint32_t o = static_cast<uint32_t>(d4);
+                float* ml = &recvML[(rank * G + row) * 2];
+                if (o == rank) {
+                    ml[0] = M;
+                    ml[1] = L;
+                } else {
+                    st_async_v2(dsmem_addr(smem_u32(ml), o), M, L, dsmem_addr(bar_merge, o));
                 }
             }
         }
-        if (C > 1) {
-            __syncthreads();
-            if (rank != 0) {
-                // every partial of this CTA is written; tell CTA 0 and leave
-                if (tid == 0) mbar_arrive_remote(dsmem_addr(smem_u32(&sm.bar_merge), 0));
-                return;
-            }
-            mbar_wait_bounded<true>(smem_u32(&sm.bar_merge), 0, p.err, 3);
-            // per (row, partial) weight exp2(m_r - M) / L: one thread per
-            // pair, reduced over the C-lane segment
-            float* fac = Ow;                   // [G][C]; the warp partials are consumed
-            merge_factors(partM, partL, G, static_cast<int>(C), fac, nullptr, nullptr, true);
-            __syncthreads();
-            for (int idx = tid; idx < G * kD; idx += kThreads) {
-                const int row = idx >> 7, d = idx & (kD - 1);
-                const float* po = partO + row * kD + d;
-                const float* fr = fac + row * C;
-                float o4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                uint32_t r = 0;
-                for (; r + 4 <= C; r += 4) {
+        // every other CTA's slice of its partial has arrived (each sends only
+        // after its own page lookups, so no CTA leaves while another may
+        // still read its staged page ids)
+        mbar_wait_bounded<true>(bar_merge, 0, p.err, 3, kWaitNs);
+        __syncthreads();                                    // this CTA's own stores
+        // merge the C partials of two channels of one row per thread
+#pragma unroll 1
+        for (int idx = tid; idx < G * ds / 2; idx += kThreads) {
+            const int row = idx >> (lgds - 1), dl = (idx & (ds / 2 - 1)) * 2;
+            float M = -INFINITY;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        o4[i] = fmaf(po[(r + i) * G * kD], fr[r + i], o4[i]);
+            for (int r = 0; r < 16; ++r)
+                if (r < static_cast<int>(C)) M = fmaxf(M, recvML[(r * G + row) * 2]);
+            float L = 0.0f, a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                if (r < static_cast<int>(C)) {
+                    const float2 ml = *reinterpret_cast<const float2*>(&recvML[(r * G + row) * 2]);
+                    const float e = M != -INFINITY ? exp2f(ml.x - M) : 0.0f;
+                    L = fmaf(ml.y, e, L);
+                    const float2 v =
+                        *reinterpret_cast<const float2*>(&recvO[(r * G + row) * ds + dl]);
+                    a0 = fmaf(v.x, e, a0);
+                    a1 = fmaf(v.y, e, a1);
                 }
-                for (; r < C; ++r) o4[0] = fmaf(po[r * G * kD], fr[r], o4[0]);
-                outp[row * kD + d] = __float2bfloat16_rn((o4[0] + o4[1]) + (o4[2] + o4[3]));
             }
+            const float rl = L > 0.0f ? 1.0f / L : 0.0f;
+            *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) =
+                pack_bf16x2(a0 * rl, a1 * rl);
         }
     }
 }
@@ -1168,11 +1305,11 @@ struct ShapeCache {
     }
 };
 
-template <int MODE, bool BIG, bool EARLY, bool BF16C, bool GM>
+template <int MODE, bool BIG, bool EARLY, bool BF16C, bool GM, bool DIAG = false>
 cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool pdl,
                         const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st,
                         bool* fits) {
-    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C, GM>;
+    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C, GM, DIAG>;
     // per device (function attributes belong to a device's context) and
     // per shape: whether one cluster of C CTAs with `smem` bytes fits
     static std::mutex mu;
@@ -1303,16 +1440,18 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     int C = pick_cluster(pairs, num_sms);
     cudaError_t e = cudaSuccess;
     for (; C >= 1; C /= 2) {
-        // region B: scores + select scratch, or this CTA's page buffers, or the
-        // warp merge; region A: code ring, or (CTA 0) the cluster merge
-        size_t regB = 0, regA = 0, scratch = 0;
+        // region B: scores + select scratch + the code ring, then this CTA's
+        // page buffers, then the warp merge; region A: the cluster merge's
+        // receive buffers
+        size_t regB = 0, regA = 0, scratch = 0, ring = 0;
         if (do_select) {
             // score slots for every row, rounded up to whole groups of 4
             scratch = (static_cast<size_t>(a.nmax + 3) / 4) * 16;
             prm.wg_off = static_cast<uint32_t>(scratch + kSelectScratch);
-            regB = std::max(regB, scratch + kSelectScratch +
-                                      (a.group_max ? static_cast<size_t>(G) * kWgStride * 4 : 0));
-            regA = std::max(regA, static_cast<size_t>(kStages) * kStageBytes);
+            const size_t used = scratch + kSelectScratch +
+                                (a.group_max ? static_cast<size_t>(G) * kWgStride * 4 : 0);
+            ring = (used + 127) & ~static_cast<size_t>(127);
+            regB = std::max(regB, ring + static_cast<size_t>(kStages) * kStageBytes);
         }
         if (do_attend) {
             // one page buffer per warp: a second one (double buffering)
@@ -1320,30 +1459,38 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
             // workload measured
             regB = std::max(regB, static_cast<size_t>(kWarps) * kPageSmem);
             regB = std::max(regB, static_cast<size_t>(kWarps) * G * (kD + 2) * 4);
-            if (C > 1) regA = std::max(regA, static_cast<size_t>(C) * G * (kD + 2) * 4);
+            // the slice merge's receive buffers: C partial slices of G x
+            // 128/C channels and (M, L) per row
+            if (C > 1)
+                regA = std::max(regA, static_cast<size_t>(G) * kD * 4 + static_cast<size_t>(8) * C * G);
         }
         regB = (regB + 1023) & ~static_cast<size_t>(1023);
         regA = (regA + 127) & ~static_cast<size_t>(127);
-        // extra code-ring stages in what region B leaves free while scoring
+        // as many ring stages as region B holds past the select scratch
         prm.nstages = kStages;
-        prm.xstage_off = 0;
-        if (do_select) {
-            const size_t used = scratch + kSelectScratch +
-                                (a.group_max ? static_cast<size_t>(G) * kWgStride * 4 : 0);
-            const size_t off = (used + 127) & ~static_cast<size_t>(127);
-            const size_t extra = regB > off ? (regB - off) / kStageBytes : 0;
-            prm.nstages = kStages + static_cast<int>(std::min<size_t>(kMaxStages - kStages, extra));
-            prm.xstage_off = static_cast<uint32_t>(off);
-        }
+        prm.ring_off = static_cast<uint32_t>(ring);
+        if (do_select)
+            prm.nstages = static_cast<int>(
+                std::min<size_t>(kMaxStages, std::max<size_t>(kStages, (regB - ring) / kStageBytes)));
         prm.scratch_off = static_cast<uint32_t>(scratch);
         prm.regA_off = static_cast<uint32_t>(regB);
         prm.small_off = static_cast<uint32_t>(regB + regA);
-        const size_t smem = 1024 + regB + regA + sizeof(Small) + static_cast<size_t>(a.kmax) * 4;
+        prm.qs_off = static_cast<uint32_t>(regB + regA + ((sizeof(Small) + 15) & ~static_cast<size_t>(15)));
+        const size_t smem =
+            1024 + prm.qs_off + static_cast<size_t>(G) * kD * 2 + static_cast<size_t>(a.kmax) * 4;
         if (smem > 227 * 1024) return cudaErrorInvalidValue;
         bool fits = false;
         const bool early = early_prefetch && mode == kModeFull;
         const bool bf = a.cfmt == ABSP_CENTROIDS_BF16, gm = a.group_max != 0;
-        if (mode == kModeAttend) {
+        if (a.diag_timeout) {
+            // the failure-path diagnostic: INT4 centroids, sum aggregation,
+            // GQA group <= 8, no early prefetch (checked by the caller)
+            e = mode == kModeSelect
+                    ? launch_mode<kModeSelect, false, false, false, false, true>(
+                          prm, smem, C, pairs, pdl, tmk, tmv, st, &fits)
+                    : launch_mode<kModeFull, false, false, false, false, true>(
+                          prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
+        } else if (mode == kModeAttend) {
             e = big ? launch_mode<kModeAttend, true, false, false, false>(
                           prm, smem, C, pairs, pdl, tmk, tmv, st, &fits)
                     : launch_mode<kModeAttend, false, false, false, false>(

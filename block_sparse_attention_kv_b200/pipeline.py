@@ -36,12 +36,18 @@ class DeviceLayer:
         self.stream = stream
 
     # -- steps 1-2 --------------------------------------------------------
-    def build_centroids(self, keep_ws: bool = False):
+    def build_centroids(self, keep_ws: bool = False, fused: bool = False):
+        """Steps 1-2: the separate build and quantize calls, or with `fused`
+        the single call (one launch when the layer's heads fit on a
+        cluster); both give the same bits."""
         if self.build_ws is None:
             n = abi.absp_build_workspace_size(self.kv)
             self.build_ws = abi.alloc_workspace(n, self.device)
-        abi.absp_build_centroids(self.kv, self.build_ws, self.stream)
-        abi.absp_quantize_centroids(self.kv, self.build_ws, self.cent, self.stream)
+        if fused:
+            abi.absp_build_quantize_centroids(self.kv, self.build_ws, self.cent, self.stream)
+        else:
+            abi.absp_build_centroids(self.kv, self.build_ws, self.stream)
+            abi.absp_quantize_centroids(self.kv, self.build_ws, self.cent, self.stream)
         self.check(self.build_ws)
         if not keep_ws:
             self.build_ws = None

@@ -175,6 +175,17 @@ ABSP_API absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws,
                                     size_t ws_bytes, const absp_centroids* out,
                                     void* stream);
 
+/* Steps 1-2 in one call, with the results of absp_build_centroids followed
+ * by absp_quantize_centroids (bit for bit), in as few passes over memory as
+ * the layer allows: when every head's centroid capacity (cap_h rows) fits
+ * on one thread-block cluster, a single launch keeps each head's fp64
+ * centroids on chip and writes only `out` (the workspace is then used for
+ * its error word alone); otherwise the two kernels of the separate calls
+ * run.  `ws` is sized by absp_build_workspace_size either way. */
+ABSP_API absp_status absp_build_quantize_centroids(const absp_layer_kv* kv, void* ws,
+                                                   size_t ws_bytes, const absp_centroids* out,
+                                                   void* stream);
+
 /* Incremental update during decode (Fig. 5: block sizes are fixed, so the
  * store is kept up to date instead of rebuilt).  Call after the caller has
  * written the new tokens' K/V into the pages and raised seq_lens.  For every
@@ -241,15 +252,30 @@ ABSP_API absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centro
  * earlier steps, the query by the kernel just before.  Without the flag
  * nothing is read before the preceding kernel has completed. */
 
-/* absp_decode_step with flags (ABSP_STEP_EARLY_PREFETCH, ABSP_STEP_GROUP_MAX;
- * other bits are rejected).  Without ABSP_STEP_GROUP_MAX, same results as
+/* ABSP_STEP_DIAG_WAIT_TIMEOUT: a diagnostic of the failure path, not a
+ * decode variant (the paper has no counterpart).  The launch runs a kernel
+ * instance whose score-exchange barrier expects 16 bytes more than the
+ * cluster sends and whose bounded waits give up after 1 ms instead of 1 s:
+ * that wait runs out, the kernel records ABSP_ERR_TIMEOUT (detail 4, the
+ * score wait) in the workspace, carries on to its normal end and returns.
+ * Its selection and output are then meaningless; the next call on the same
+ * workspace, after absp_check_device_error has read and cleared the error
+ * word, runs normally.  Only with INT4 centroids, sum aggregation, a GQA
+ * group of at most 8 and without ABSP_STEP_EARLY_PREFETCH
+ * (ABSP_ERR_UNSUPPORTED otherwise). */
+#define ABSP_STEP_DIAG_WAIT_TIMEOUT 0x100u
+
+/* absp_decode_step with flags (ABSP_STEP_EARLY_PREFETCH, ABSP_STEP_GROUP_MAX,
+ * ABSP_STEP_DIAG_WAIT_TIMEOUT; other bits are rejected).  Without
+ * ABSP_STEP_GROUP_MAX and the diagnostic, same results as
  * absp_decode_step. */
 ABSP_API absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                          const void* q, int32_t budget_tokens, void* out,
                                          void* ws, size_t ws_bytes, uint32_t flags,
                                          void* stream);
 
-/* absp_score_select with flags (0 or ABSP_STEP_GROUP_MAX). */
+/* absp_score_select with flags (0, ABSP_STEP_GROUP_MAX or
+ * ABSP_STEP_DIAG_WAIT_TIMEOUT). */
 ABSP_API absp_status absp_score_select_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                           const void* q, int32_t budget_tokens, int32_t* sel,
                                           int32_t* sel_count, void* ws, size_t ws_bytes,
