@@ -754,6 +754,24 @@ def gpu_arm(args):
         append = {"us_per_layer": ms_a / (args.steps * L) * 1e3,
                   "note": "absp_append_centroids, all 8 KV heads of one layer per launch"}
         del ga
+        # the decode loop's own order: each layer's centroid tail update,
+        # then its decode step, which may then read nothing before the
+        # update completes (the plain step, no early prefetch)
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            for x in layers:
+                abi.absp_append_centroids(x.kv, x.cent, None, x.ws, sc)
+                abi.absp_decode_step(x.kv, x.cent, x.data.q, x.budget, x.out, x.ws, sc)
+        with torch.cuda.stream(stream):
+            ms_ad = timed(gd, args.steps, args.warmup)
+        for x in layers:
+            x.check()
+        append["then_decode"] = {
+            "value": aggregate_rate(world, L, args.steps, ms_ad),
+            "us_per_layer": ms_ad / (args.steps * L) * 1e3,
+            "note": "per layer: absp_append_centroids then absp_decode_step (plain), the "
+                    "sequence a decode loop runs; layer-steps/s"}
+        del gd
 
     # fixed block size for every KV head (the uniform-block methods the page
     # compares against) and unquantised bf16 centroids (its precision

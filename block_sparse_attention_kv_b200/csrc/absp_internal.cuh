@@ -141,6 +141,20 @@ __device__ __forceinline__ void mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 // ------------------------------------------------------- async copies --
 
+// 4-byte asynchronous copy global -> shared (no register staging); completed
+// by cp_async_wait_all() in the issuing thread.
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 // 1-D bulk copy global -> this CTA's shared memory; completes `bytes` of
 // transaction count on `bar`.  16-byte aligned addresses, size % 16 == 0.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
@@ -150,6 +164,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         "[%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// Fetch a tensor-map descriptor (a __grid_constant__ kernel parameter) into
+// the copy engine's descriptor cache ahead of its first use.
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // 2-D tensor tile load (no multicast) into this CTA's shared memory.

@@ -88,6 +88,8 @@ struct Params {
     uint32_t wg_off;              // per-head weights inside region B
     int32_t nstages;              // code ring stages (kStages .. kMaxStages)
     uint32_t ring_off;            // code ring inside region B, past the select scratch
+    uint32_t ptrow_off;           // staged page-table row, after the list
+    int32_t pt_cap;               // entries the staged row holds (0: none)
 };
 
 // per-head score weights for the group-max variant: [G][8 lanes][20]
@@ -113,14 +115,31 @@ struct Small {                    // fixed-size shared scratch
     alignas(16) uint32_t scan[kWarps];
 };
 
+// 2^x by the hardware approximation (relative error ~2^-22, far inside
+// the bf16 output; -inf gives +0), and a hardware reciprocal.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t order_key(float f) {
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // Monotone (non-decreasing) map of a score onto kBins bins of [mn, mx].
+// (x - mn) * inv >= 0 for x >= mn; adding 2^23 rounding toward zero puts
+// its integer part in the low mantissa bits (an ALU floor, no conversion).
 __device__ __forceinline__ int value_bin(float x, float mn, float inv) {
-    return __float2int_rz(fminf((x - mn) * inv, static_cast<float>(kBins - 1)));
+    const float y = fminf((x - mn) * inv, static_cast<float>(kBins - 1));
+    return __float_as_int(__fadd_rz(y, 8388608.0f)) - 0x4B000000;
 }
 
 __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) {
@@ -298,11 +317,11 @@ __device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int
 // Top-k of sc[0..n) (largest scores, ties to the lower index) in ascending
 // index order; only list entries [lo, hi) are written, to out[0 .. hi-lo).
 // [mn, mx] is the range of the scores.  The kBins histogram bins at the
-// start of `scratch` must be zero on entry.  n <= 65535.
-template <typename OnBoundary>
+// start of `scratch` must be zero on entry.  n <= 65535.  Ends with a block
+// barrier.
 __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float mn, float mx,
                                            int32_t* out, int lo, int hi, uint32_t* scratch,
-                                           Small& sm, OnBoundary&& on_boundary) {
+                                           Small& sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (k >= n) {
         for (int i = max(0, lo) + tid; i < min(n, hi); i += kThreads) out[i - lo] = i;
@@ -313,7 +332,9 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
     uint32_t* ckey = scratch + kBins;
     int32_t* cidx = reinterpret_cast<int32_t*>(scratch + kBins + kMaxCand);
     uint32_t* inw = scratch + kBins + 2 * kMaxCand;
-    const float inv = static_cast<float>(kBins) / (mx - mn);
+    // any monotone binning that every CTA computes alike is exact here (the
+    // K-th score's bin is then ranked exactly), so a fast division will do
+    const float inv = __fdividef(static_cast<float>(kBins), mx - mn);
     if (!(mx > mn)) {                 // every score equal: lowest k indices
         compact_by_threshold(sc, n, order_key(mx), k, out, lo, hi, sm);
         return;
@@ -375,7 +396,6 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
         }
         __syncthreads();
         const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
-        on_boundary(bstar, mn, inv);
         if (m <= kMaxCand) {
             // one pass: a ballot word per 32 scores marks those above bin
             // bstar (selected); the scores inside bstar become candidates,
@@ -394,6 +414,8 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                     x[v] = jb == j0 ? kx[v] : (live ? sc[i] : mn);
                     bnv[v] = jb == j0 ? kbin[v] : (live ? value_bin(x[v], mn, inv) : -1);
                 }
+                uint32_t cw[V];     // candidates (scores in bin bstar) of each word
+                uint32_t ncand = 0;
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     const int wd = jb + v;
@@ -404,10 +426,24 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                         __ballot_sync(0xffffffffu, live && (bn > bstar || (all_in && bn == bstar)));
                     if (lane == 0 && wd < j1) inw[wd] = gw;
                     cnt += __popc(gw);
-                    if (!all_in && live && bn == bstar) {
-                        const int pos = atomicAdd(&sm.misc[3], 1);
-                        ckey[pos] = order_key(x[v]);
-                        cidx[pos] = i;
+                    cw[v] = all_in ? 0u : __ballot_sync(0xffffffffu, live && bn == bstar);
+                    ncand += __popc(cw[v]);
+                }
+                if (ncand != 0) {
+                    // one slot reservation per warp and chunk, then each
+                    // candidate lane writes at its place
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&sm.misc[3], static_cast<int>(ncand));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        if ((cw[v] >> lane) & 1u) {
+                            const int pos = base + __popc(cw[v] & lt);
+                            ckey[pos] = order_key(x[v]);
+                            cidx[pos] = (jb + v) * 32 + lane;
+                        }
+                        base += __popc(cw[v]);
                     }
                 }
             }
@@ -501,6 +537,15 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     constexpr int kSRows = kStageBytes / kRow;         // rows per bulk stage
     constexpr uint64_t kWaitNs = DIAG ? 1000000ull : kWaitLimitNs;
 
+    if constexpr (kAttend) {
+        // the page copies' tensor-map descriptors, fetched ahead of the
+        // first copy (they are kernel parameters, not produced by the
+        // preceding kernel)
+        if (tid == 32) {
+            prefetch_tensormap(&tmk);
+            prefetch_tensormap(&tmv);
+        }
+    }
     if (tid == 0) {
         for (int i = 0; i < kMaxStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
         for (int w = 0; w < kWarps; ++w) mbar_init(smem_u32(&sm.bar_page[w]), 1);
@@ -534,7 +579,17 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     // cluster is still running: none leaves before it received every other
     // CTA's merge partial).  Uniform over a cluster.
     const int Ksel = min(n, max(1, p.budget >> lgbs));
-    const bool stage_pt = kSelect && kAttend && per > 0 && per * spb <= kPtStage &&
+    // Preferred: every CTA stages the sequence's whole page-table row in its
+    // own shared memory (asynchronous 4-byte copies issued here, before the
+    // dependency wait with early prefetch), so that a page id is one local
+    // read.  When the row does not fit, the own-rows slices below.
+    int32_t* ptrow = reinterpret_cast<int32_t*>(base + p.ptrow_off);
+    const bool stage_row = kSelect && kAttend && npg <= p.pt_cap;
+    if (stage_row) {
+        for (int i = tid; i < npg; i += kThreads) cp_async_4(smem_u32(ptrow + i), pt + i);
+        cp_async_commit();
+    }
+    const bool stage_pt = kSelect && kAttend && !stage_row && per > 0 && per * spb <= kPtStage &&
                           ((Ksel * spb + static_cast<int>(C) - 1) >> lgC) <= 32 * kWarps;
     int ptv[kPtStage / kThreads];
 #pragma unroll
@@ -576,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     // B0 arrive (release: the barrier set-up above is visible cluster-wide
     // once B0 completes); matched by the wait before the first remote access.
     cluster_arrive();
-    if (kAttend && !stage_pt) {
+    if (kAttend && !stage_pt && !stage_row) {
         // the attention phase reads page-table entries of this sequence
         for (int i = tid * 32; i < npg; i += kThreads * 32) prefetch_l2(pt + i);
     }
@@ -588,6 +643,14 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             scl = p.scale[pi];
             zpv = p.zp[pi];
         }
+    }
+    if constexpr (EARLY && kSelect) {
+        // an L2 hint for the group's queries (read below, after the wait;
+        // when the preceding kernel writes them, its writes land in L2 and
+        // the read sees them, as it would without this hint)
+        if (tid < G * kD * 2 / 128)
+            prefetch_l2(reinterpret_cast<const uint8_t*>(
+                            p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD) + tid * 128);
     }
     if constexpr (EARLY) {
         // B0 only needs the cluster's CTAs to have started: wait for it while
@@ -607,6 +670,8 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
 #pragma unroll
             for (int u = 0; u < kPtStage / kThreads; ++u) sm.pt[tid + u * kThreads] = ptv[u];
         }
+        if (stage_row) cp_async_wait_all();   // this thread's copies; the barrier below
+                                              // makes the whole row visible
         if (tid < kD) {
             const __nv_bfloat16* qh = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD + tid;
             // the group's queries are read once (they may live in host
@@ -856,47 +921,32 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         mbar_wait_bounded<true>(bar_score, 0, p.err, 4, kWaitNs);
 
         // --------------------------------------------------- C: select --
-        float smin = INFINITY, smax = -INFINITY;
+        float2 rv[16];                       // C <= 16: a tree, not a chain
 #pragma unroll
-        for (uint32_t r = 0; r < 16; ++r) {  // C <= 16; independent loads
-            if (r < C) {
-                smin = fminf(smin, sm.cmm[r].x);
-                smax = fmaxf(smax, sm.cmm[r].y);
+        for (uint32_t r = 0; r < 16; ++r) rv[r] = r < C ? sm.cmm[r] : make_float2(INFINITY, -INFINITY);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+            for (int r = 0; r < w; ++r) {
+                rv[r].x = fminf(rv[r].x, rv[r + w].x);
+                rv[r].y = fmaxf(rv[r].y, rv[r + w].y);
             }
         }
+        const float smin = rv[0].x, smax = rv[0].y;
+        // this CTA attends list entries [sel_lo, sel_hi): the blocks of its
+        // share [ppb, ppe) of the K * bs/16 selected pages
+        const int Pp = K * spb;
+        const int ppb = static_cast<int>((static_cast<uint32_t>(Pp) * rank) >> lgC);  // P*C < 2^21
+        const int ppe = static_cast<int>((static_cast<uint32_t>(Pp) * (rank + 1)) >> lgC);
         if (MODE == kModeSelect) {
             sel_lo = 0;
             sel_hi = K;
         } else {
-            // this CTA attends list entries [sel_lo, sel_hi): the blocks of
-            // its share [pb, pe) of the K * bs/16 selected pages
-            const int P = K * spb;
-            const int pb = static_cast<int>((static_cast<uint32_t>(P) * rank) >> lgC);  // P*C < 2^21
-            const int pe = static_cast<int>((static_cast<uint32_t>(P) * (rank + 1)) >> lgC);
-            sel_lo = pb >> lgspb;
-            sel_hi = pe > pb ? ((pe - 1) >> lgspb) + 1 : sel_lo;
+            sel_lo = ppb >> lgspb;
+            sel_hi = ppe > ppb ? ((ppe - 1) >> lgspb) + 1 : sel_lo;
         }
-        // once the boundary bin is known, the pages of this CTA's own rows
-        // that score above it (selected whatever the boundary ranking gives)
-        // start their way into L2 while the selection is finished
-        auto prefetch_sure = [&](int bstar, float mn, float inv) {
-            if constexpr (kAttend) {
-                if (!stage_pt) return;
-                for (int r = tid; r < nrows; r += kThreads) {
-                    if (value_bin(scores[r0 + r], mn, inv) <= bstar) continue;
-                    for (int jj = 0; jj < spb; ++jj) {
-                        const int lp = (r0 + r) * spb + jj;
-                        const int phys = sm.pt[r * spb + jj];
-                        if (lp >= npg || phys < 0 || phys >= p.kv.num_phys_pages) break;
-                        const int64_t off = (static_cast<int64_t>(phys) * Hkv + h) * (kPage * kD);
-                        bulk_prefetch_l2(p.kv.k_pages + off, kPage * kD * 2);
-                        bulk_prefetch_l2(p.kv.v_pages + off, kPage * kD * 2);
-                    }
-                }
-            }
-        };
         block_topk(scores, n, K, smin, smax, sel_s, sel_lo, sel_hi,
-                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm, prefetch_sure);
+                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm);
         if (MODE == kModeSelect) {
             int32_t* dst = p.sel + (static_cast<int64_t>(s) * Hkv + h) * p.kmax;
             for (int i = tid; i < K; i += kThreads) dst[i] = sel_s[i];  // [0, K) held
@@ -965,7 +1015,9 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             const int valid = min(kPage, len - lp * kPage);
             if (valid <= 0) return;
             int phys;
-            if (stage_pt) {
+            if (stage_row) {
+                phys = ptrow[lp];
+            } else if (stage_pt) {
                 // staged by the CTA that scored block b
                 // b / per by a float reciprocal, corrected to the exact
                 // quotient (b < 2^14, per >= 4)
@@ -1021,7 +1073,8 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             bulk_prefetch_l2(p.kv.v_pages + off, kPage * kD * 2);
         };
 
-        __syncthreads();  // every thread is done with the scores in region B
+        // (the select, or the copy of a given selection, ended with a barrier:
+        // no thread reads the scores in region B any more)
         resolve(0);
         int vnext = cnt_w > 0 ? issue(0) : 0;
 #pragma unroll 1
@@ -1083,9 +1136,9 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                 // valid >= 1 so token 0 is valid: mx is finite
                 const float mn0 = fmaxf(m0, mx);
-                const float corr0 = any0 ? exp2f(m0 - mn0) : 0.0f;
-                const uint32_t pa0 = pack_bf16x2(exp2f(x0 - mn0), exp2f(x1 - mn0));
-                const uint32_t pa2 = pack_bf16x2(exp2f(x2 - mn0), exp2f(x3 - mn0));
+                const float corr0 = any0 ? fast_exp2(m0 - mn0) : 0.0f;
+                const uint32_t pa0 = pack_bf16x2(fast_exp2(x0 - mn0), fast_exp2(x1 - mn0));
+                const uint32_t pa2 = pack_bf16x2(fast_exp2(x2 - mn0), fast_exp2(x3 - mn0));
                 l0 = l0 * corr0 + (bf16lo(pa0) + bf16hi(pa0) + bf16lo(pa2) + bf16hi(pa2));
                 m0 = mn0;
                 uint32_t pa1 = 0u, pa3 = 0u;
@@ -1099,22 +1152,24 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                     my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, 1));
                     my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, 2));
                     const float mn8 = fmaxf(m8, my);
-                    corr8 = any0 ? exp2f(m8 - mn8) : 0.0f;
-                    pa1 = pack_bf16x2(exp2f(y0 - mn8), exp2f(y1 - mn8));
-                    pa3 = pack_bf16x2(exp2f(y2 - mn8), exp2f(y3 - mn8));
+                    corr8 = any0 ? fast_exp2(m8 - mn8) : 0.0f;
+                    pa1 = pack_bf16x2(fast_exp2(y0 - mn8), fast_exp2(y1 - mn8));
+                    pa3 = pack_bf16x2(fast_exp2(y2 - mn8), fast_exp2(y3 - mn8));
                     l8 = l8 * corr8 + (bf16lo(pa1) + bf16hi(pa1) + bf16lo(pa3) + bf16hi(pa3));
                     m8 = mn8;
                 }
-                any0 = true;
+                if (any0) {   // nothing to rescale before this warp's first valid page
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    o[t][0] *= corr0;
-                    o[t][1] *= corr0;
-                    if constexpr (BIG_GROUP) {
-                        o[t][2] *= corr8;
-                        o[t][3] *= corr8;
+                    for (int t = 0; t < 16; ++t) {
+                        o[t][0] *= corr0;
+                        o[t][1] *= corr0;
+                        if constexpr (BIG_GROUP) {
+                            o[t][2] *= corr8;
+                            o[t][3] *= corr8;
+                        }
                     }
                 }
+                any0 = true;
                 // O[row][d] += P[row][token] V[token][d]
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
@@ -1134,9 +1189,11 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                     }
                 }
             }
-            fence_proxy_async_smem();  // this lane's reads/writes of the buffer
-            __syncwarp();              // before its next tensor copy
-            if (i + 1 < cnt_w) vnext = issue(i + 1);
+            if (i + 1 < cnt_w) {
+                fence_proxy_async_smem();  // this lane's reads/writes of the buffer
+                __syncwarp();              // before its next tensor copy
+                vnext = issue(i + 1);
+            }
             if (ABSP_PAGE_PREFETCH > 0) prefetch(i + 1 + ABSP_PAGE_PREFETCH);
         }
         l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -1199,7 +1256,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
-                const float e = M != -INFINITY ? exp2f(mv[w] - M) : 0.0f;
+                const float e = M != -INFINITY ? fast_exp2(mv[w] - M) : 0.0f;
                 L = fmaf(lw[w * G + row], e, L);
                 const float4 v = *reinterpret_cast<const float4*>(&Ow[(w * G + row) * kD + d]);
                 a.x = fmaf(v.x, e, a.x);
@@ -1215,7 +1272,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                 const int row = idx / (kD / 4), d = (idx % (kD / 4)) * 4;
                 float M, L;
                 const float4 a = cta_partial(row, d, M, L);
-                const float r = L > 0.0f ? 1.0f / L : 0.0f;
+                const float r = L > 0.0f ? fast_rcp(L) : 0.0f;
                 // 4-byte stores: the output is only 4-byte aligned
                 uint32_t* o2 = reinterpret_cast<uint32_t*>(outp + row * kD + d);
                 o2[0] = pack_bf16x2(a.x * r, a.y * r);
@@ -1256,30 +1313,42 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         // still read its staged page ids)
         mbar_wait_bounded<true>(bar_merge, 0, p.err, 3, kWaitNs);
         __syncthreads();                                    // this CTA's own stores
-        // merge the C partials of two channels of one row per thread
-#pragma unroll 1
+        // per (row, partial) weight exp2(M_r - M) / L: one thread per pair
+        // (G * C <= 256), the C partials of a row on C consecutive lanes
+        // reduced by shuffles; then two channels of one row per thread
+        float* fac = reinterpret_cast<float*>(regB);   // [G][C]; the warp partials are consumed
+        {
+            const int pairs = G << lgC;
+            if (tid < ((pairs + 31) & ~31)) {             // whole warps (full-mask shuffles)
+                const bool act = tid < pairs;
+                const int row = act ? tid >> lgC : 0, r = act ? tid & (static_cast<int>(C) - 1) : 0;
+                const float2 ml = act ? *reinterpret_cast<const float2*>(&recvML[(r * G + row) * 2])
+                                      : make_float2(-INFINITY, 0.0f);
+                float M = ml.x;
+                for (int o = 1; o < static_cast<int>(C); o <<= 1)
+                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+                const float e = M != -INFINITY ? fast_exp2(ml.x - M) : 0.0f;
+                float L = ml.y * e;
+                for (int o = 1; o < static_cast<int>(C); o <<= 1)
+                    L += __shfl_xor_sync(0xffffffffu, L, o);
+                if (act) fac[(row << lgC) + r] = L > 0.0f ? e * fast_rcp(L) : 0.0f;
+            }
+        }
+        __syncthreads();
         for (int idx = tid; idx < G * ds / 2; idx += kThreads) {
             const int row = idx >> (lgds - 1), dl = (idx & (ds / 2 - 1)) * 2;
-            float M = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r < static_cast<int>(C)) M = fmaxf(M, recvML[(r * G + row) * 2]);
-            float L = 0.0f, a0 = 0.0f, a1 = 0.0f;
+            const float* fr = fac + (row << lgC);
+            float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 if (r < static_cast<int>(C)) {
-                    const float2 ml = *reinterpret_cast<const float2*>(&recvML[(r * G + row) * 2]);
-                    const float e = M != -INFINITY ? exp2f(ml.x - M) : 0.0f;
-                    L = fmaf(ml.y, e, L);
                     const float2 v =
                         *reinterpret_cast<const float2*>(&recvO[(r * G + row) * ds + dl]);
-                    a0 = fmaf(v.x, e, a0);
-                    a1 = fmaf(v.y, e, a1);
+                    a0 = fmaf(v.x, fr[r], a0);
+                    a1 = fmaf(v.y, fr[r], a1);
                 }
             }
-            const float rl = L > 0.0f ? 1.0f / L : 0.0f;
-            *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) =
-                pack_bf16x2(a0 * rl, a1 * rl);
+            *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) = pack_bf16x2(a0, a1);
         }
     }
 }
@@ -1476,8 +1545,18 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
         prm.regA_off = static_cast<uint32_t>(regB);
         prm.small_off = static_cast<uint32_t>(regB + regA);
         prm.qs_off = static_cast<uint32_t>(regB + regA + ((sizeof(Small) + 15) & ~static_cast<size_t>(15)));
-        const size_t smem =
-            1024 + prm.qs_off + static_cast<size_t>(G) * kD * 2 + static_cast<size_t>(a.kmax) * 4;
+        // the fused step stages whole page-table rows in what is left of a
+        // two-CTAs-per-SM share of shared memory (rows that do not fit use
+        // the per-CTA slices or global reads)
+        const size_t tail = (static_cast<size_t>(prm.qs_off) + static_cast<size_t>(G) * kD * 2 +
+                             static_cast<size_t>(a.kmax) * 4 + 15) & ~static_cast<size_t>(15);
+        prm.ptrow_off = static_cast<uint32_t>(tail);
+        prm.pt_cap = 0;
+        constexpr size_t kTwoPerSm = 112 * 1024;
+        if (do_select && do_attend && 1024 + tail < kTwoPerSm)
+            prm.pt_cap = static_cast<int32_t>(
+                std::min<size_t>(a.kv.max_pages, (kTwoPerSm - 1024 - tail) / 4) & ~static_cast<size_t>(3));
+        const size_t smem = 1024 + tail + static_cast<size_t>(prm.pt_cap) * 4;
         if (smem > 227 * 1024) return cudaErrorInvalidValue;
         bool fits = false;
         const bool early = early_prefetch && mode == kModeFull;
