@@ -1335,20 +1335,34 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             }
         }
         __syncthreads();
-        for (int idx = tid; idx < G * ds / 2; idx += kThreads) {
-            const int row = idx >> (lgds - 1), dl = (idx & (ds / 2 - 1)) * 2;
+        // two channels of one row per 4 consecutive lanes, each lane summing
+        // every 4th partial, then a 2-step shuffle: each output takes C/4
+        // dependent steps instead of C
+        const int tot = G * ds * 2;
+        for (int base = 0; base < tot; base += kThreads) {
+            if (base + (tid & ~31) >= tot) break;     // whole warps (full-mask shuffles)
+            const int idx = base + tid;
+            const bool act = idx < tot;
+            const int pr = act ? idx >> 2 : 0, qtr = idx & 3;
+            const int row = pr >> (lgds - 1), dl = (pr & (ds / 2 - 1)) * 2;
             const float* fr = fac + (row << lgC);
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                if (r < static_cast<int>(C)) {
+            for (int r4 = 0; r4 < 16; r4 += 4) {
+                const int r = r4 + qtr;
+                if (act && r < static_cast<int>(C)) {
                     const float2 v =
                         *reinterpret_cast<const float2*>(&recvO[(r * G + row) * ds + dl]);
                     a0 = fmaf(v.x, fr[r], a0);
                     a1 = fmaf(v.y, fr[r], a1);
                 }
             }
-            *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) = pack_bf16x2(a0, a1);
+            a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+            a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+            if (act && qtr == 0)
+                *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) = pack_bf16x2(a0, a1);
         }
     }
 }
