@@ -56,6 +56,24 @@ __device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
     return v;
 }
 
+// x / cnt for a block's token count: a power of two (every full block) is
+// an exact scaling by its reciprocal; a ragged tail divides.
+__device__ __forceinline__ double mean_of(double x, int cnt, double inv_pow2) {
+    return (cnt & (cnt - 1)) == 0 ? x * inv_pow2 : x / static_cast<double>(cnt);
+}
+
+// rint(c / sc) (IEEE division, round half to even) without dividing on the
+// common path: r = c * inv (inv = 1 / sc rounded) is within 2^-51 |c/sc| of
+// the quotient, so unless r lies within 2^-48 max(|r|, 1) of a half-integer
+// (where rint could jump) its rint is the quotient's; otherwise divide.
+__device__ __forceinline__ double rint_div(double c, double sc, double inv) {
+    const double r = c * inv;
+    const double fl = floor(r);
+    const double d = r - fl;
+    if (fabs(d - 0.5) <= fmax(fabs(r), 1.0) * 0x1p-48) return rint(c / sc);
+    return d > 0.5 ? fl + 1.0 : fl;
+}
+
 // Validated sequence length; faults are recorded once per sequence.
 __device__ __forceinline__ int checked_len(const KvDesc& kv, int s, int32_t* err) {
     const int len = kv.seq_lens[s];
@@ -139,12 +157,13 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
                 }
             }
         }
-        const double dc = static_cast<double>(cnt);
+        // 2^-k for cnt = 2^k (used only then)
+        const double dinv = __hiloint2double((1023 - (__ffs(cnt) - 1)) << 20, 0);
         double2* dg = reinterpret_cast<double2*>(cent + static_cast<int64_t>(b) * kD + hl * 8);
         double2* ds = reinterpret_cast<double2*>(&rows_s[b - b_begin][hl * 8]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const double2 c = make_double2(a[2 * i] / dc, a[2 * i + 1] / dc);
+            const double2 c = make_double2(mean_of(a[2 * i], cnt, dinv), mean_of(a[2 * i + 1], cnt, dinv));
             dg[i] = c;
             ds[i] = c;
         }
@@ -226,11 +245,12 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
     const int b_begin = tok0 / bs;
     const int b_end = min(n, (tok0 + kChunkTokens) / bs);
     const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h];
-    double sc[4], zz[4];
+    double sc[4], zz[4], iv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         sc[i] = s_scale[lane * 4 + i];
         zz[i] = s_zp[lane * 4 + i];
+        iv[i] = sc[i] != 0.0 ? 1.0 / sc[i] : 0.0;
     }
     for (int b = b_begin + warp; b < b_end; b += kBuildWarps) {
         const double2* src = reinterpret_cast<const double2*>(w.cent + (row0 + b) * kD + lane * 4);
@@ -241,7 +261,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
         for (int i = 0; i < 4; ++i) {
             uint32_t code = 0;
             if (sc[i] != 0.0) {
-                double qv = rint(c[i] / sc[i]) + zz[i];
+                double qv = rint_div(c[i], sc[i], iv[i]) + zz[i];
                 qv = fmin(fmax(qv, 0.0), 15.0);
                 code = static_cast<uint32_t>(qv);
             }
@@ -482,10 +502,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
             }
         }
-        const double dc = static_cast<double>(cnt);
+        // 2^-k for cnt = 2^k (used only then)
+        const double dinv = __hiloint2double((1023 - (__ffs(cnt) - 1)) << 20, 0);
         double2* dst = reinterpret_cast<double2*>(cent + static_cast<size_t>(r) * kD + hl * 8);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_double2(a[2 * i] / dc, a[2 * i + 1] / dc);
+        for (int i = 0; i < 4; ++i)
+            dst[i] = make_double2(mean_of(a[2 * i], cnt, dinv), mean_of(a[2 * i + 1], cnt, dinv));
     }
     __syncthreads();
 
@@ -582,12 +604,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---- store: INT4 codes (4 bytes per lane) or bf16 rows (16 bytes)
     const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h] + r0;
-    double sc[8], zz[8];
+    double sc[8], zz[8], iv[8];
     if (int4) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             sc[i] = par[hl * 8 + i];
             zz[i] = par[kD + hl * 8 + i];
+            iv[i] = sc[i] != 0.0 ? 1.0 / sc[i] : 0.0;
         }
     }
     for (int r = hw; r < nrows; r += kFusedHalfWarps) {
@@ -605,7 +628,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             for (int i = 0; i < 8; ++i) {
                 uint32_t code = 0;
                 if (sc[i] != 0.0) {
-                    double qv = rint(c[i] / sc[i]) + zz[i];
+                    double qv = rint_div(c[i], sc[i], iv[i]) + zz[i];
                     qv = fmin(fmax(qv, 0.0), 15.0);
                     code = static_cast<uint32_t>(qv);
                 }
