@@ -332,10 +332,8 @@ cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st);
 cudaError_t launch_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
                             int32_t* zp, int format, cudaStream_t st);
 
-// Steps 1-2 in as few launches as the layer allows: one fused cluster
-// kernel when every head's centroids fit on a cluster, else build + quantize
-// (centroids.cu).  `w` is used for its error word, and fully by the
-// two-pass path.
+// Steps 1-2 in one call (centroids.cu): the build kernel and the quantise
+// kernel (INT4), or the build kernel writing bf16 rows directly (BF16).
 cudaError_t launch_build_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
                                   int32_t* zp, int format, cudaStream_t st);
 

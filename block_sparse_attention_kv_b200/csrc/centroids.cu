@@ -74,6 +74,141 @@ __device__ __forceinline__ double rint_div(double c, double sc, double inv) {
     return d > 0.5 ? fl + 1.0 : fl;
 }
 
+// ---------------------------------------------------------------------------
+// Exact block sums of bf16 keys.
+//
+// The centroid of a block is the token-order fp64 sum of its keys over the
+// token count.  That sum is exact, and so equal to the sum in any order,
+// whenever the block's nonzero values span few enough binades: a bf16 value
+// with biased exponent e is a multiple of 2^(e-134) below 2^(e-126), so with
+// exponents in [emin, emax] and at most 64 tokens every partial sum is a
+// multiple of 2^(emin-134) below 2^(emax-120), and fp64 holds it exactly
+// when emax - emin <= 39.  Under that condition a page's 16 rows may be
+// summed in any exact way.  The fast path sums them in fp32 twice, rounded
+// down and rounded up: each rounded sum bounds the exact one from its side
+// (also through further additions of such bounds, each rounded the same
+// way), so where the two agree both are exact.  One fp32 -> fp64 conversion
+// per page and channel then replaces sixteen.  A page whose two sums differ
+// is summed in fp64 instead; a block that fails the exponent condition (or
+// holds a zero, subnormal, infinite or NaN key) is summed again in token
+// order, as the definition reads.
+
+// One word of a key row (two bf16 keys, channels c and c+1) into the
+// fast path's state: both keys widened to fp32 and added to the round-down
+// and round-up sums (packed pairs, low channel first), and the keys'
+// magnitudes (bf16 bits without the sign, as 16-bit integers: ordered as
+// the values' magnitudes, NaN above infinity) folded into the running
+// min / max.  One asm block, so that each word is consumed as it arrives.
+__device__ __forceinline__ void fold_word(uint64_t& dn, uint64_t& up, uint32_t& mn, uint32_t& mx,
+                                          uint32_t w) {
+    asm("{\n\t"
+        ".reg .b32 lo, hi, m;\n\t"
+        ".reg .b64 f;\n\t"
+        "shl.b32 lo, %4, 16;\n\t"
+        "and.b32 hi, %4, 0xFFFF0000;\n\t"
+        "mov.b64 f, {lo, hi};\n\t"
+        "add.rm.f32x2 %0, %0, f;\n\t"
+        "add.rp.f32x2 %1, %1, f;\n\t"
+        "and.b32 m, %4, 0x7FFF7FFF;\n\t"
+        "min.u16x2 %2, %2, m;\n\t"
+        "max.u16x2 %3, %3, m;\n\t"
+        "}"
+        : "+l"(dn), "+l"(up), "+r"(mn), "+r"(mx)
+        : "r"(w));
+}
+
+__device__ __forceinline__ float f32x2_lo(uint64_t v) {
+    return __uint_as_float(static_cast<uint32_t>(v));
+}
+
+__device__ __forceinline__ float f32x2_hi(uint64_t v) {
+    return __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+
+// Channels 8hl .. 8hl+7 of a block's cnt keys summed into a[] (pages[j]
+// is the block's j-th page), bit-identical to the token-order fp64 sums.
+// The first pass takes the fast path page by page; a page whose two fp32
+// sums differ is read again and added to a[] in fp64 token by token (exact
+// under the exponent condition, checked at the end).  If the condition
+// fails, a second pass sums the block in token order throughout.  Both
+// passes share one load site, so the rare branches hold no registers of
+// their own.
+__device__ __forceinline__ void block_sums(const KvDesc& kv, const int32_t* pages, int h, int hl,
+                                           int cnt, int s, int32_t* err, double a[8]) {
+    bool ordered = false;   // second pass: the definition, term by term
+    for (;;) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = 0.0;
+        uint32_t mn = 0xFFFFFFFFu, mx = 0u;   // |key| extremes over the block, 16-bit pairs
+        for (int j = 0; j * kPage < cnt; ++j) {
+            const int nt = min(kPage, cnt - j * kPage);
+            const int phys = pages[j];
+            if (phys < 0 || phys >= kv.num_phys_pages) {
+                if (hl == 0) set_error(err, ABSP_ERR_DEVICE_FAULT, s);
+                continue;
+            }
+            const __nv_bfloat16* src =
+                kv.k_pages + ((static_cast<int64_t>(phys) * kv.Hkv + h) * kPage) * kD + hl * 8;
+            bool slow = ordered;
+            for (;;) {
+                uint4 v[kPage];
+#pragma unroll
+                for (int t = 0; t < kPage; ++t)
+                    if (t < nt) v[t] = ld_nc_u4(src + t * kD);
+                if (slow) {
+#pragma unroll
+                    for (int t = 0; t < kPage; ++t) {
+                        if (t < nt) {
+                            a[0] += static_cast<double>(bf16lo(v[t].x));
+                            a[1] += static_cast<double>(bf16hi(v[t].x));
+                            a[2] += static_cast<double>(bf16lo(v[t].y));
+                            a[3] += static_cast<double>(bf16hi(v[t].y));
+                            a[4] += static_cast<double>(bf16lo(v[t].z));
+                            a[5] += static_cast<double>(bf16hi(v[t].z));
+                            a[6] += static_cast<double>(bf16lo(v[t].w));
+                            a[7] += static_cast<double>(bf16hi(v[t].w));
+                        }
+                    }
+                    break;
+                }
+                uint64_t dn[4] = {0, 0, 0, 0}, up[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int t = 0; t < kPage; ++t) {
+                    if (t < nt) {
+                        fold_word(dn[0], up[0], mn, mx, v[t].x);
+                        fold_word(dn[1], up[1], mn, mx, v[t].y);
+                        fold_word(dn[2], up[2], mn, mx, v[t].z);
+                        fold_word(dn[3], up[3], mn, mx, v[t].w);
+                    }
+                }
+                bool exact = true;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    exact = exact && f32x2_lo(dn[i]) == f32x2_lo(up[i]) &&
+                            f32x2_hi(dn[i]) == f32x2_hi(up[i]);
+                if (exact) {
+                    // the round-up sums: +0 where an exact sum is zero, as in fp64
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        a[2 * i] += static_cast<double>(f32x2_lo(up[i]));
+                        a[2 * i + 1] += static_cast<double>(f32x2_hi(up[i]));
+                    }
+                    break;
+                }
+                slow = true;
+            }
+        }
+        if (ordered) return;
+        const int emin = static_cast<int>(min(mn & 0xFFFFu, mn >> 16) >> 7);
+        const int emax = static_cast<int>(max(mx & 0xFFFFu, mx >> 16) >> 7);
+        bool ok = emin >= 1 && emax <= 254 && emax - emin <= 39;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ok = ok && a[i] == a[i];
+        if (ok) return;
+        ordered = true;
+    }
+}
+
 // Validated sequence length; faults are recorded once per sequence.
 __device__ __forceinline__ int checked_len(const KvDesc& kv, int s, int32_t* err) {
     const int len = kv.seq_lens[s];
@@ -96,16 +231,18 @@ __device__ __forceinline__ uint32_t f64_to_bf16_rne(double x) {
     return u >> 16;
 }
 
-// Two-pass build: one CTA per (1024-token chunk, KV head, sequence).  Each
-// half-warp takes one block at a time; lane l (of 16) owns channels
-// 8l .. 8l+7 and reads 16 bytes of every key row (a half-warp reads a whole
-// 256-byte row per instruction, a page's 16 rows in flight).  Token-order
-// fp64 sums.  The chunk's centroids go to the workspace and to shared
-// memory; the CTA's per-channel min / max is taken over the shared copy and
-// merged with one atomic per channel into order-mapped keys (the max as the
-// key of its negation, so that one fill of ones initialises every key).
+// One 1024-token chunk of (sequence s, KV head h), by one CTA of
+// kBuildWarps warps.  Each half-warp takes one block at a time; lane l (of
+// 16) owns channels 8l .. 8l+7 and reads 16 bytes of every key row (a
+// half-warp reads a whole 256-byte row per instruction, a page's 16 rows in
+// flight).  Sums as block_sums.  With bf16_rows the centroids are stored
+// there rounded to bf16 and nothing else is done; otherwise they go to the
+// workspace and to shared memory, and the chunk's per-channel min / max,
+// taken over the shared copy, is merged with one atomic per channel into
+// order-mapped keys (the max as the key of its negation, so that one fill
+// of ones initialises every key).
 __global__ void __launch_bounds__(kBuildWarps * 32)
-    centroid_build_kernel(const KvDesc kv, BuildWs w) {
+    centroid_build_kernel(const KvDesc kv, BuildWs w, uint8_t* __restrict__ bf16_rows) {
     const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x;
     const int hw = tid >> 4, hl = tid & 15;            // half-warp, lane within it
@@ -122,52 +259,37 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
     const int b_begin = tok0 / bs;
     const int b_end = min(n, (tok0 + kChunkTokens) / bs);
     const int32_t* pt = kv.page_table + static_cast<int64_t>(s) * kv.max_pages;
-    double* cent = w.cent + (static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h]) * kD;
+    const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h];
 
     for (int b = b_begin + hw; b < b_end; b += kHalfWarps) {
         const int t0 = b * bs;
         const int cnt = min(bs, len - t0);
         double a[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = 0.0;
-        for (int tp = t0; tp < t0 + cnt; tp += kPage) {
-            const int nt = min(kPage, t0 + cnt - tp);
-            const int phys = pt[tp / kPage];
-            if (phys < 0 || phys >= kv.num_phys_pages) {
-                if (hl == 0) set_error(w.err, ABSP_ERR_DEVICE_FAULT, s);
-                continue;
-            }
-            const __nv_bfloat16* src =
-                kv.k_pages + ((static_cast<int64_t>(phys) * kv.Hkv + h) * kPage) * kD + hl * 8;
-            uint4 v[kPage];
-#pragma unroll
-            for (int t = 0; t < kPage; ++t)
-                if (t < nt) v[t] = ld_nc_u4(src + t * kD);
-#pragma unroll
-            for (int t = 0; t < kPage; ++t) {
-                if (t < nt) {
-                    a[0] += static_cast<double>(bf16lo(v[t].x));
-                    a[1] += static_cast<double>(bf16hi(v[t].x));
-                    a[2] += static_cast<double>(bf16lo(v[t].y));
-                    a[3] += static_cast<double>(bf16hi(v[t].y));
-                    a[4] += static_cast<double>(bf16lo(v[t].z));
-                    a[5] += static_cast<double>(bf16hi(v[t].z));
-                    a[6] += static_cast<double>(bf16lo(v[t].w));
-                    a[7] += static_cast<double>(bf16hi(v[t].w));
-                }
-            }
-        }
+        block_sums(kv, pt + t0 / kPage, h, hl, cnt, s, w.err, a);
         // 2^-k for cnt = 2^k (used only then)
         const double dinv = __hiloint2double((1023 - (__ffs(cnt) - 1)) << 20, 0);
-        double2* dg = reinterpret_cast<double2*>(cent + static_cast<int64_t>(b) * kD + hl * 8);
+        double c[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) c[i] = mean_of(a[i], cnt, dinv);
+        if (bf16_rows != nullptr) {
+            uint4 o;
+            o.x = f64_to_bf16_rne(c[0]) | (f64_to_bf16_rne(c[1]) << 16);
+            o.y = f64_to_bf16_rne(c[2]) | (f64_to_bf16_rne(c[3]) << 16);
+            o.z = f64_to_bf16_rne(c[4]) | (f64_to_bf16_rne(c[5]) << 16);
+            o.w = f64_to_bf16_rne(c[6]) | (f64_to_bf16_rne(c[7]) << 16);
+            *reinterpret_cast<uint4*>(bf16_rows + (row0 + b) * (2 * kD) + hl * 16) = o;
+            continue;
+        }
+        double2* dg = reinterpret_cast<double2*>(w.cent + (row0 + b) * kD + hl * 8);
         double2* ds = reinterpret_cast<double2*>(&rows_s[b - b_begin][hl * 8]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const double2 c = make_double2(mean_of(a[2 * i], cnt, dinv), mean_of(a[2 * i + 1], cnt, dinv));
-            dg[i] = c;
-            ds[i] = c;
+            const double2 v = make_double2(c[2 * i], c[2 * i + 1]);
+            dg[i] = v;
+            ds[i] = v;
         }
     }
+    if (bf16_rows != nullptr) return;  // uniform
     __syncthreads();
     // per-channel min / max of the chunk's rows: thread t takes channel
     // t % 128 of every other row, the two halves merged by one shuffle-free
@@ -196,19 +318,53 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
     }
 }
 
+// Quantise: one CTA per (group of `rows_per_cta` rows, a multiple of 32 up
+// to kQuantRows, KV head, sequence), launched as a programmatic dependent
+// of the build so that it is resident when the build ends; it waits for
+// the build's results before reading them.  Threads 0..127 derive the
+// per-channel parameters (fp64 divisions) while the first rows' loads are
+// in flight.  Warp w codes rows w, w + 8, ...
+// of the group four at a time, the next four's loads issued before the
+// current four are coded; lane L takes channels 4L .. 4L+3 and writes 2
+// bytes of each 64-byte row.
+constexpr int kQuantRows = 256;
+
 __global__ void __launch_bounds__(kBuildWarps * 32)
     centroid_quantize_kernel(const KvDesc kv, BuildWs w, uint8_t* __restrict__ codes,
-                             float* __restrict__ scale_out, int32_t* __restrict__ zp_out) {
-    const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+                             float* __restrict__ scale_out, int32_t* __restrict__ zp_out,
+                             int rows_per_cta) {
+    const int grp = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ double s_scale[kD];
-    __shared__ double s_zp[kD];
+    __shared__ double s_par[3][kD];   // scale, zero point, 1 / scale
 
     const int len = checked_len(kv, s, w.err);
-    const int tok0 = chunk * kChunkTokens;
-    if (chunk > 0 && len <= tok0) return;  // uniform over the CTA
     const int bs = kv.bs[h];
     const int n = len > 0 ? (len + bs - 1) / bs : 0;
+    const int r_begin = grp * rows_per_cta;
+    if (grp > 0 && r_begin >= n) return;  // uniform over the CTA
+    const int r_end = min(n, r_begin + rows_per_cta);
+    pdl_wait();                           // the build's rows and keys
+    const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h];
+
+    constexpr int kRows = 4;
+    constexpr int kStep = kRows * kBuildWarps;
+    double c0[kRows][4], c1[kRows][4];
+    auto load = [&](int b0, double (&cb)[kRows][4]) {
+#pragma unroll
+        for (int q = 0; q < kRows; ++q) {
+            const int b = b0 + q * kBuildWarps;
+            if (b < r_end) {
+                const double2* src =
+                    reinterpret_cast<const double2*>(w.cent + (row0 + b) * kD + lane * 4);
+                const double2 u = src[0], v = src[1];
+                cb[q][0] = u.x;
+                cb[q][1] = u.y;
+                cb[q][2] = v.x;
+                cb[q][3] = v.y;
+            }
+        }
+    };
+    load(r_begin + warp, c0);
 
     if (threadIdx.x < kD) {
         const int d = threadIdx.x;
@@ -232,43 +388,49 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
                 }
             }
         }
-        s_scale[d] = sc;
-        s_zp[d] = z;
-        if (chunk == 0) {
+        s_par[0][d] = sc;
+        s_par[1][d] = z;
+        s_par[2][d] = sc != 0.0 ? 1.0 / sc : 0.0;
+        if (grp == 0) {
             scale_out[pi] = scf;
             zp_out[pi] = zi;
         }
     }
     __syncthreads();
-    if (len <= tok0) return;
-
-    const int b_begin = tok0 / bs;
-    const int b_end = min(n, (tok0 + kChunkTokens) / bs);
-    const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h];
     double sc[4], zz[4], iv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        sc[i] = s_scale[lane * 4 + i];
-        zz[i] = s_zp[lane * 4 + i];
-        iv[i] = sc[i] != 0.0 ? 1.0 / sc[i] : 0.0;
+        sc[i] = s_par[0][lane * 4 + i];
+        zz[i] = s_par[1][lane * 4 + i];
+        iv[i] = s_par[2][lane * 4 + i];
     }
-    for (int b = b_begin + warp; b < b_end; b += kBuildWarps) {
-        const double2* src = reinterpret_cast<const double2*>(w.cent + (row0 + b) * kD + lane * 4);
-        const double2 u = src[0], v = src[1];
-        const double c[4] = {u.x, u.y, v.x, v.y};
-        uint32_t packed = 0;
+    auto code_rows = [&](int b0, const double (&cb)[kRows][4]) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t code = 0;
-            if (sc[i] != 0.0) {
-                double qv = rint_div(c[i], sc[i], iv[i]) + zz[i];
-                qv = fmin(fmax(qv, 0.0), 15.0);
-                code = static_cast<uint32_t>(qv);
+        for (int q = 0; q < kRows; ++q) {
+            const int b = b0 + q * kBuildWarps;
+            if (b >= r_end) break;
+            uint32_t packed = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t code = 0;
+                if (sc[i] != 0.0) {
+                    double qv = rint_div(cb[q][i], sc[i], iv[i]) + zz[i];
+                    qv = fmin(fmax(qv, 0.0), 15.0);
+                    code = static_cast<uint32_t>(qv);
+                }
+                packed |= code << (4 * i);
             }
-            packed |= code << (4 * i);
+            *reinterpret_cast<uint16_t*>(codes + (row0 + b) * kRowBytes + lane * 2) =
+                static_cast<uint16_t>(packed);
         }
-        *reinterpret_cast<uint16_t*>(codes + (row0 + b) * kRowBytes + lane * 2) =
-            static_cast<uint16_t>(packed);
+    };
+    // two buffers, named, so that every index is static
+    for (int b0 = r_begin + warp; b0 < r_end; b0 += 2 * kStep) {
+        if (b0 + kStep < r_end) load(b0 + kStep, c1);
+        code_rows(b0, c0);
+        if (b0 + kStep >= r_end) break;
+        if (b0 + 2 * kStep < r_end) load(b0 + 2 * kStep, c0);
+        code_rows(b0 + kStep, c1);
     }
 }
 
@@ -381,277 +543,16 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
 }
 
 
-// ---------------------------------------------------------------------------
-// Steps 1-2 in one launch: one thread-block cluster of C CTAs per
-// (sequence, KV head) keeps the head's fp64 centroids in shared memory, so
-// nothing goes through global memory but the keys read and the codes
-// written.
-//   build:    CTA r takes a contiguous 1/C of the head's blocks; each
-//             half-warp takes one block at a time, lane l (of 16) owns
-//             channels 8l .. 8l+7 and reads 16 bytes of every key row (a
-//             half-warp reads a whole 256-byte row per instruction, the 16
-//             rows of a page in flight at once).  Token-order fp64 sums, as
-//             in the two-pass build.  Each CTA's per-channel min / max:
-//             across the two half-warps of a warp by shuffle, across warps
-//             by shared-memory atomics on order-mapped keys.
-//   exchange: every CTA sends its 128 mins and 128 maxes to every CTA of
-//             the cluster (16-byte asynchronous stores counted on the
-//             receiver's mbarrier); all CTAs then hold the head's min / max
-//             and derive the same scale / zero point.
-//   quantize: every CTA codes its own rows from shared memory.
-// A head fits when its centroid capacity is at most C x kFusedRows rows; a
-// layer with a larger head takes the two-pass kernels.
-constexpr int kFusedThreads = 512;
-constexpr int kFusedHalfWarps = kFusedThreads / 16;
-constexpr int kFusedRows = 160;                 // fp64 centroid rows per CTA
-
-
-__device__ __forceinline__ void st_async_u4(uint32_t remote_addr, uint4 v, uint32_t remote_bar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, "
-        "[%5];" ::"r"(remote_addr),
-        "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
-        : "memory");
-}
-
-__global__ void __launch_bounds__(kFusedThreads, 1)
-    centroid_fused_kernel(const KvDesc kv, int32_t* err, int rows_cap, uint8_t* __restrict__ codes,
-                          float* __restrict__ scale_out, int32_t* __restrict__ zp_out,
-                          int format) {
-    extern __shared__ __align__(16) uint8_t fsm[];
-    const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
-    const int pair = blockIdx.x / C;
-    const int s = pair / kv.Hkv, h = pair % kv.Hkv;
-    const int tid = threadIdx.x;
-    const int hw = tid >> 4, hl = tid & 15;      // half-warp, lane within it
-    const bool int4 = format != ABSP_CENTROIDS_BF16;
-    double* cent = reinterpret_cast<double*>(fsm);                            // [rows_cap][128]
-    double* recv = cent + static_cast<size_t>(rows_cap) * kD;                 // [C][2][128]
-    unsigned long long* red = reinterpret_cast<unsigned long long*>(recv + C * 2 * kD);  // [2][128]
-    double* par = reinterpret_cast<double*>(red + 2 * kD);                   // scale, zp [2][128]
-    int32_t* pg = reinterpret_cast<int32_t*>(par + 2 * kD);                   // [rows_cap * 4]
-    unsigned long long* bar = reinterpret_cast<unsigned long long*>(pg + rows_cap * 4);
-    const uint32_t bar_a = smem_u32(bar);
-
-    if (tid == 0) {
-        mbar_init(bar_a, 1);
-        fence_mbar_init();
-        // every other CTA's 128 mins and 128 maxes
-        if (int4 && C > 1) mbar_arrive_expect_tx(bar_a, (C - 1) * 2 * kD * 8);
-    }
-    if (tid < kD) {
-        red[tid] = ~0ull;        // min keys
-        red[kD + tid] = 0ull;    // max keys
-    }
-    // release: the barrier set-up is visible cluster-wide once the matching
-    // wait (before the first remote store) completes
-    cluster_arrive();
-
-    int len = kv.seq_lens[s];
-    if (len < 0 || len > kv.max_pages * kPage) {
-        if (tid == 0 && rank == 0 && h == 0) set_error(err, ABSP_ERR_DEVICE_FAULT, s);
-        len = 0;
-    }
-    const int bs = kv.bs[h];
-    const int spb = bs / kPage;
-    const int n = (len + bs - 1) / bs;
-    const int per = (n + static_cast<int>(C) - 1) / static_cast<int>(C);  // <= rows_cap
-    const int r0 = min(n, static_cast<int>(rank) * per);
-    const int nrows = min(n, r0 + per) - r0;
-    const int npg = (len + kPage - 1) / kPage;
-    // page ids of this CTA's blocks, read once, in parallel
-    const int32_t* pt = kv.page_table + static_cast<int64_t>(s) * kv.max_pages;
-    for (int i = tid; i < nrows * spb; i += kFusedThreads) {
-        const int lp = r0 * spb + i;
-        pg[i] = lp < npg ? pt[lp] : -1;
-    }
-    __syncthreads();
-
-    // ---- build: token-order fp64 sums, one block per half-warp at a time
-    for (int r = hw; r < nrows; r += kFusedHalfWarps) {
-        const int b = r0 + r;
-        const int t0 = b * bs;
-        const int cnt = min(bs, len - t0);
-        double a[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = 0.0;
-        for (int j = 0; j * kPage < cnt; ++j) {
-            const int nt = min(kPage, cnt - j * kPage);
-            const int phys = pg[r * spb + j];
-            if (phys < 0 || phys >= kv.num_phys_pages) {
-                if (hl == 0) set_error(err, ABSP_ERR_DEVICE_FAULT, s);
-                continue;
-            }
-            const __nv_bfloat16* src =
-                kv.k_pages + ((static_cast<int64_t>(phys) * kv.Hkv + h) * kPage) * kD + hl * 8;
-            uint4 v[kPage];
-#pragma unroll
-            for (int t = 0; t < kPage; ++t)
-                if (t < nt) v[t] = ld_nc_u4(src + t * kD);
-#pragma unroll
-            for (int t = 0; t < kPage; ++t) {
-                if (t < nt) {
-                    a[0] += static_cast<double>(bf16lo(v[t].x));
-                    a[1] += static_cast<double>(bf16hi(v[t].x));
-                    a[2] += static_cast<double>(bf16lo(v[t].y));
-                    a[3] += static_cast<double>(bf16hi(v[t].y));
-                    a[4] += static_cast<double>(bf16lo(v[t].z));
-                    a[5] += static_cast<double>(bf16hi(v[t].z));
-                    a[6] += static_cast<double>(bf16lo(v[t].w));
-                    a[7] += static_cast<double>(bf16hi(v[t].w));
-                }
-            }
-        }
-        // 2^-k for cnt = 2^k (used only then)
-        const double dinv = __hiloint2double((1023 - (__ffs(cnt) - 1)) << 20, 0);
-        double2* dst = reinterpret_cast<double2*>(cent + static_cast<size_t>(r) * kD + hl * 8);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            dst[i] = make_double2(mean_of(a[2 * i], cnt, dinv), mean_of(a[2 * i + 1], cnt, dinv));
-    }
-    __syncthreads();
-
-    if (int4) {
-        // ---- this CTA's per-channel min / max over its rows in shared
-        // memory (thread t: channel t % 128, every 4th row), then the
-        // cluster's
-        {
-            const int d = tid & (kD - 1), q4 = tid >> 7;
-            double mn = __longlong_as_double(0x7FF0000000000000ll), mx = -mn;
-            for (int r = q4; r < nrows; r += kFusedThreads / kD) {
-                const double c = cent[static_cast<size_t>(r) * kD + d];
-                mn = fmin(mn, c);
-                mx = fmax(mx, c);
-            }
-            if (mn <= mx) {
-                atomicMin(&red[d], ord_f64(mn));
-                atomicMax(&red[kD + d], ord_f64(mx));
-            }
-        }
-        __syncthreads();
-        cluster_wait();   // every CTA's barrier is initialised
-        // 256 doubles (mins, then maxes) = 128 pieces of 16 bytes to every
-        // CTA; a CTA with no block sends the +inf / -inf sentinels
-        for (int i = tid; i < static_cast<int>(C) * 128; i += kFusedThreads) {
-            const uint32_t dst_rank = static_cast<uint32_t>(i / 128);
-            const int piece = i % 128;
-            const int k0 = 2 * piece;
-            auto val = [&](int k) -> double {
-                const unsigned long long key = red[k];
-                if (k < kD ? key == ~0ull : key == 0ull)
-                    return k < kD ? __longlong_as_double(0x7FF0000000000000ll)
-                                  : __longlong_as_double(static_cast<long long>(0xFFF0000000000000ull));
-                return unord_f64(key);
-            };
-            const double d0 = val(k0), d1 = val(k0 + 1);
-            double* slot = recv + (rank * 2) * kD + k0;
-            if (dst_rank == rank) {
-                slot[0] = d0;
-                slot[1] = d1;
-            } else {
-                uint4 u;
-                u.x = static_cast<uint32_t>(__double_as_longlong(d0));
-                u.y = static_cast<uint32_t>(static_cast<unsigned long long>(__double_as_longlong(d0)) >> 32);
-                u.z = static_cast<uint32_t>(__double_as_longlong(d1));
-                u.w = static_cast<uint32_t>(static_cast<unsigned long long>(__double_as_longlong(d1)) >> 32);
-                st_async_u4(dsmem_addr(smem_u32(slot), dst_rank), u, dsmem_addr(bar_a, dst_rank));
-            }
-        }
-        if (C > 1) {
-            // bounded wait: every other CTA's (min, max) has arrived
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait_cluster(bar_a, 0)) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    set_error(err, ABSP_ERR_TIMEOUT, 6);
-                    break;
-                }
-            }
-        }
-        __syncthreads();
-        if (tid < kD) {
-            const int d = tid;
-            double lo = recv[d], hi = recv[kD + d];
-            for (uint32_t r = 1; r < C; ++r) {
-                lo = fmin(lo, recv[(2 * r) * kD + d]);
-                hi = fmax(hi, recv[(2 * r + 1) * kD + d]);
-            }
-            double sc = 0.0, z = 0.0;
-            float scf = 0.0f;
-            int32_t zi = 0;
-            if (n > 0 && hi > lo) {
-                const float f = __double2float_rn((hi - lo) / 15.0);
-                if (f > 0.0f) {
-                    scf = f;
-                    sc = static_cast<double>(f);
-                    double zr = rint(-lo / sc);
-                    zr = fmin(fmax(zr, -2147483648.0), 2147483647.0);
-                    zi = static_cast<int32_t>(zr);
-                    z = static_cast<double>(zi);
-                }
-            }
-            par[d] = sc;
-            par[kD + d] = z;
-            if (rank == 0) {
-                const int64_t pi = (static_cast<int64_t>(s) * kv.Hkv + h) * kD + d;
-                scale_out[pi] = scf;
-                zp_out[pi] = zi;
-            }
-        }
-    } else {
-        cluster_wait();
-    }
-    __syncthreads();
-
-    // ---- store: INT4 codes (4 bytes per lane) or bf16 rows (16 bytes)
-    const int64_t row0 = static_cast<int64_t>(s) * kv.rows_per_seq + kv.row_base[h] + r0;
-    double sc[8], zz[8], iv[8];
-    if (int4) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            sc[i] = par[hl * 8 + i];
-            zz[i] = par[kD + hl * 8 + i];
-            iv[i] = sc[i] != 0.0 ? 1.0 / sc[i] : 0.0;
-        }
-    }
-    for (int r = hw; r < nrows; r += kFusedHalfWarps) {
-        const double2* src = reinterpret_cast<const double2*>(cent + static_cast<size_t>(r) * kD + hl * 8);
-        double c[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const double2 u = src[i];
-            c[2 * i] = u.x;
-            c[2 * i + 1] = u.y;
-        }
-        if (int4) {
-            uint32_t packed = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                uint32_t code = 0;
-                if (sc[i] != 0.0) {
-                    double qv = rint_div(c[i], sc[i], iv[i]) + zz[i];
-                    qv = fmin(fmax(qv, 0.0), 15.0);
-                    code = static_cast<uint32_t>(qv);
-                }
-                packed |= code << (4 * i);
-            }
-            *reinterpret_cast<uint32_t*>(codes + (row0 + r) * kRowBytes + hl * 4) = packed;
-        } else {
-            uint4 o;
-            o.x = f64_to_bf16_rne(c[0]) | (f64_to_bf16_rne(c[1]) << 16);
-            o.y = f64_to_bf16_rne(c[2]) | (f64_to_bf16_rne(c[3]) << 16);
-            o.z = f64_to_bf16_rne(c[4]) | (f64_to_bf16_rne(c[5]) << 16);
-            o.w = f64_to_bf16_rne(c[6]) | (f64_to_bf16_rne(c[7]) << 16);
-            *reinterpret_cast<uint4*>(codes + (row0 + r) * (2 * kD) + hl * 16) = o;
-        }
-    }
-}
-
 }  // namespace
 
+// [header][min / max keys][fp64 rows]
+static size_t minmax_bytes(const KvDesc& kv) {
+    return static_cast<size_t>(kv.S) * kv.Hkv * kD * 2 * sizeof(unsigned long long);
+}
+
 size_t build_ws_bytes(const KvDesc& kv) {
-    const size_t mm = static_cast<size_t>(kv.S) * kv.Hkv * kD * 2 * sizeof(unsigned long long);
     const size_t cent = static_cast<size_t>(kv.S) * kv.rows_per_seq * kD * sizeof(double);
-    return kWsHeader + mm + cent;
+    return kWsHeader + minmax_bytes(kv) + cent;
 }
 
 BuildWs build_ws_layout(void* ws, const KvDesc& kv) {
@@ -659,8 +560,7 @@ BuildWs build_ws_layout(void* ws, const KvDesc& kv) {
     BuildWs w;
     w.err = reinterpret_cast<int32_t*>(p);
     w.minmax = reinterpret_cast<unsigned long long*>(p + kWsHeader);
-    const size_t mm = static_cast<size_t>(kv.S) * kv.Hkv * kD * 2 * sizeof(unsigned long long);
-    w.cent = reinterpret_cast<double*>(p + kWsHeader + mm);
+    w.cent = reinterpret_cast<double*>(p + kWsHeader + minmax_bytes(kv));
     return w;
 }
 
@@ -669,12 +569,14 @@ static dim3 chunk_grid(const KvDesc& kv) {
     return dim3(chunks, kv.Hkv, kv.S);
 }
 
-cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st) {
-    // order-mapped sentinels: every key (min of c, and min of -c for the
-    // max) starts at all-ones
-    const size_t pairs = static_cast<size_t>(kv.S) * kv.Hkv * kD;
-    cudaError_t e = cudaMemsetAsync(w.minmax, 0xFF, 2 * pairs * sizeof(unsigned long long), st);
-    if (e != cudaSuccess) return e;
+// The build kernel, writing fp64 rows + min / max keys (after one fill of
+// ones over the keys), or, with bf16_rows, bf16 rows only.
+static cudaError_t launch_build_rows(const KvDesc& kv, const BuildWs& w, uint8_t* bf16_rows,
+                                     cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
+    if (bf16_rows == nullptr &&
+        (e = cudaMemsetAsync(w.minmax, 0xFF, minmax_bytes(kv), st)) != cudaSuccess)
+        return e;
     static std::mutex mu;
     static bool configured[16] = {};
     int dev = 0;
@@ -694,8 +596,13 @@ cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st) {
         cudaThreadExchangeStreamCaptureMode(&mode);
         if (e != cudaSuccess) return e;
     }
-    centroid_build_kernel<<<chunk_grid(kv), kBuildWarps * 32, kBuildSmem, st>>>(kv, w);
+    centroid_build_kernel<<<chunk_grid(kv), kBuildWarps * 32, bf16_rows ? 0 : kBuildSmem, st>>>(
+        kv, w, bf16_rows);
     return cudaGetLastError();
+}
+
+cudaError_t launch_build(const KvDesc& kv, const BuildWs& w, cudaStream_t st) {
+    return launch_build_rows(kv, w, nullptr, st);
 }
 
 cudaError_t launch_append(const KvDesc& kv, uint8_t* codes, const float* scale, const int32_t* zp,
@@ -708,78 +615,39 @@ cudaError_t launch_append(const KvDesc& kv, uint8_t* codes, const float* scale, 
 
 cudaError_t launch_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
                             int32_t* zp, int format, cudaStream_t st) {
-    if (format == ABSP_CENTROIDS_BF16)
+    if (format == ABSP_CENTROIDS_BF16) {
         centroid_bf16_kernel<<<chunk_grid(kv), kBuildWarps * 32, 0, st>>>(kv, w, codes);
-    else
-        centroid_quantize_kernel<<<chunk_grid(kv), kBuildWarps * 32, 0, st>>>(kv, w, codes, scale,
-                                                                           zp);
+    } else {
+        // rows per CTA: enough CTAs to fill the GPU a few times over, each
+        // with whole 32-row steps
+        int cap = 1, dev = 0, num_sms = 148;
+        for (int h = 0; h < kv.Hkv; ++h) cap = std::max(cap, kv.cap[h]);
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            num_sms = 148;
+        const long long rows = static_cast<long long>(kv.S) * kv.rows_per_seq;
+        const long long want = (rows / (4ll * num_sms) + 31) / 32 * 32;
+        const int rpc = static_cast<int>(std::min<long long>(kQuantRows, std::max(32ll, want)));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((cap + rpc - 1) / rpc, kv.Hkv, kv.S);
+        cfg.blockDim = dim3(kBuildWarps * 32);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, centroid_quantize_kernel, kv, w, codes, scale, zp, rpc);
+    }
     return cudaGetLastError();
 }
 
 
-size_t fused_smem_bytes(int rows_cap, int C) {
-    return static_cast<size_t>(rows_cap) * kD * 8 + static_cast<size_t>(C) * 2 * kD * 8 +
-           2 * kD * 8 + 2 * kD * 8 + static_cast<size_t>(rows_cap) * 4 * 4 + 16;
-}
-
-// Cluster size of the fused build, or 0 when some head's centroids do not
-// fit on one cluster (the two-pass kernels then run instead).
-int fused_cluster(const KvDesc& kv, int num_sms, int* rows_cap) {
-    int cap = 0;
-    for (int h = 0; h < kv.Hkv; ++h) cap = std::max(cap, kv.cap[h]);
-    int C = 1;
-    while (C < 16 && (cap + C - 1) / C > kFusedRows) C *= 2;
-    if ((cap + C - 1) / C > kFusedRows) return 0;
-    const int pairs = kv.S * kv.Hkv;
-    // more CTAs per head while the launch still fits in one wave
-    while (C < 16 && pairs * C * 2 <= num_sms) C *= 2;
-    *rows_cap = (cap + C - 1) / C;
-    return C;
-}
-
 cudaError_t launch_build_quantize(const KvDesc& kv, const BuildWs& w, uint8_t* codes, float* scale,
                                   int32_t* zp, int format, cudaStream_t st) {
-    static std::mutex mu;
-    static bool configured[16] = {};
-    int dev = 0, num_sms = 148;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        num_sms = 148;
-    int rows_cap = 0;
-    int C = fused_cluster(kv, num_sms, &rows_cap);
-    if (C > 0) {
-        cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
-        cudaThreadExchangeStreamCaptureMode(&mode);
-        {
-            std::lock_guard<std::mutex> lock(mu);
-            if (dev < 0 || dev >= 16 || !configured[dev]) {
-                e = cudaFuncSetAttribute(centroid_fused_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-                if (e == cudaSuccess)
-                    e = cudaFuncSetAttribute(centroid_fused_kernel,
-                                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-                if (e == cudaSuccess && dev >= 0 && dev < 16) configured[dev] = true;
-            }
-        }
-        cudaThreadExchangeStreamCaptureMode(&mode);
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(kv.S * kv.Hkv * C);
-        cfg.blockDim = dim3(kFusedThreads);
-        cfg.dynamicSmemBytes = fused_smem_bytes(rows_cap, C);
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, centroid_fused_kernel, kv, w.err, rows_cap, codes, scale,
-                                  zp, format);
-    }
-    e = launch_build(kv, w, st);
+    // BF16: the build writes the rows itself, one launch
+    if (format == ABSP_CENTROIDS_BF16) return launch_build_rows(kv, w, codes, st);
+    cudaError_t e = launch_build(kv, w, st);
     if (e != cudaSuccess) return e;
     return launch_quantize(kv, w, codes, scale, zp, format, st);
 }

@@ -38,8 +38,7 @@ class DeviceLayer:
     # -- steps 1-2 --------------------------------------------------------
     def build_centroids(self, keep_ws: bool = False, fused: bool = False):
         """Steps 1-2: the separate build and quantize calls, or with `fused`
-        the single call (one launch when the layer's heads fit on a
-        cluster); both give the same bits."""
+        the single call; both give the same bits."""
         if self.build_ws is None:
             n = abi.absp_build_workspace_size(self.kv)
             self.build_ws = abi.alloc_workspace(n, self.device)

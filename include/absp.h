@@ -136,8 +136,9 @@ ABSP_API absp_status absp_centroid_sizes_fmt(const absp_layer_kv* kv, int32_t fo
 ABSP_API absp_status absp_centroid_row_offset(const absp_layer_kv* kv, int32_t seq,
                                      int32_t kv_head, int64_t* row);
 
-/* Workspace bytes for absp_build_centroids + absp_quantize_centroids:
- * 256 B header + per-channel min/max + fp64 centroids (1 KiB per row). */
+/* Workspace bytes for absp_build_centroids + absp_quantize_centroids (and
+ * absp_build_quantize_centroids): 256 B header + per-channel min/max +
+ * fp64 centroids (1 KiB per row). */
 ABSP_API absp_status absp_build_workspace_size(const absp_layer_kv* kv, size_t* bytes);
 
 /* Workspace bytes for the decode calls (score/select, sparse decode,
@@ -159,7 +160,16 @@ ABSP_API absp_status absp_workspace_init(void* ws, size_t ws_bytes, void* stream
  * valid keys, c[b][ch] = (sum_t K[t][ch]) / cnt_b, summed in token order in
  * fp64 (a ragged last block averages its valid tokens only).  Writes the
  * fp64 centroids and the per-channel min/max into `ws` (size from
- * absp_build_workspace_size).  Reads every key of the layer once. */
+ * absp_build_workspace_size).  Reads every key of the layer once.
+ * Layout of `ws` afterwards: a 256-byte header (the error word), then
+ * S * Hkv * 128 * 2 order-mapped 8-byte min / max keys, then the fp64
+ * centroids, 128 doubles per row, block b of (seq, kv_head) at row
+ * absp_centroid_row_offset(seq, kv_head) + b.
+ * The sums are exact whenever a block's nonzero keys span at most 39
+ * binades, so the kernel may add them in any exact way (fp32 page sums
+ * proved exact by rounding down and up); blocks outside that condition,
+ * or holding a zero, subnormal, infinite or NaN key, are summed in token
+ * order.  The results are the token-order sums either way. */
 ABSP_API absp_status absp_build_centroids(const absp_layer_kv* kv, void* ws,
                                  size_t ws_bytes, void* stream);
 
@@ -176,12 +186,10 @@ ABSP_API absp_status absp_quantize_centroids(const absp_layer_kv* kv, void* ws,
                                     void* stream);
 
 /* Steps 1-2 in one call, with the results of absp_build_centroids followed
- * by absp_quantize_centroids (bit for bit), in as few passes over memory as
- * the layer allows: when every head's centroid capacity (cap_h rows) fits
- * on one thread-block cluster, a single launch keeps each head's fp64
- * centroids on chip and writes only `out` (the workspace is then used for
- * its error word alone); otherwise the two kernels of the separate calls
- * run.  `ws` is sized by absp_build_workspace_size either way. */
+ * by absp_quantize_centroids (bit for bit): for INT4 those two steps'
+ * launches; for BF16 one launch of the build kernel writing the bf16 rows
+ * directly (no fp64 rows, no min / max).  `ws` is sized by
+ * absp_build_workspace_size. */
 ABSP_API absp_status absp_build_quantize_centroids(const absp_layer_kv* kv, void* ws,
                                                    size_t ws_bytes, const absp_centroids* out,
                                                    void* stream);

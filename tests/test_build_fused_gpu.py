@@ -1,7 +1,7 @@
 """Steps 1-2 in one call (absp_build_quantize_centroids) against the two
 separate calls, bit for bit, and against the oracle on the full
-Llama-shaped layer.  Layers whose heads fit on a cluster take the fused
-one-launch kernel; the large rebuild layer falls back to the two kernels."""
+Llama-shaped layer; heads up to 8192 rows (one 128K sequence at block
+size 16).  The BF16 store takes one launch that writes the rows directly."""
 
 import numpy as np
 import pytest
@@ -54,9 +54,9 @@ def test_fused_equals_two_calls(lib, w, fmt):
         assert torch.equal(a.cent.zp, b.cent.zp)
 
 
-def test_fused_falls_back_for_heads_too_large_for_a_cluster(lib):
+def test_fused_on_heads_of_8192_rows(lib):
     abi, pipeline = lib
-    # one 128K sequence with block size 16: 8192 rows, more than a cluster keeps
+    # one 128K sequence with block size 16: 8192 rows in one head
     w = synth.custom("fused_fallback", 1, 8, 2, [131072], [16, 64], 2048, seed=43)
     d = synth.make_layer(w, 0, "cuda")
     a = pipeline.DeviceLayer(d)
