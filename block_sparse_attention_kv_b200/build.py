@@ -27,10 +27,13 @@ LIB = os.path.join(LIBDIR, "libabsp.so")
 SOURCES = ["abi.cu", "centroids.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["absp_internal.cuh", "absp_trace.h"]
 
-STAMP = LIB + ".build_id"
+# a second build for profiling only: the decode kernel records phase stamps
+# (ABSP_PHASE_STAMPS); the product library never carries them
+LIB_STAMPS = os.path.join(LIBDIR, "libabsp_stamps.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17"]
+STAMP_FLAGS = ["-DABSP_PHASE_STAMPS"]
 
 
 def nvcc() -> str:
@@ -40,7 +43,7 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found (set NVCC or install the CUDA toolkit)")
 
 
-def source_hash() -> str:
+def source_hash(extra_flags=()) -> str:
     """SHA-256 (first 16 hex digits) of everything the library is built
     from: the CUDA sources and headers, the public header, this script and
     the compile flags.  It is compiled into the library (absp_build_id) and
@@ -53,32 +56,36 @@ def source_hash() -> str:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
             h.update(f.read())
-    h.update(" ".join(ARCH + FLAGS).encode())
+    h.update(" ".join(ARCH + FLAGS + list(extra_flags)).encode())
     return h.hexdigest()[:16]
 
 
-def built_id() -> str:
-    """Build id recorded beside the library at its last build ('' if none)."""
+def built_id(lib: str = LIB) -> str:
+    """Build id recorded beside a library at its last build ('' if none)."""
     try:
-        with open(STAMP) as f:
+        with open(lib + ".build_id") as f:
             return f.read().strip()
     except OSError:
         return ""
 
 
-def _stale(want: str) -> bool:
-    return not os.path.exists(LIB) or built_id() != want
+def _stale(want: str, lib: str = LIB) -> bool:
+    return not os.path.exists(lib) or built_id(lib) != want
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+def build(force: bool = False, verbose_ptxas: bool = False, stamps: bool = False) -> str:
     """Compile the library unless the one in place was built from exactly
-    the current sources (same source hash); return its path."""
-    want = source_hash()
-    if not force and not verbose_ptxas and not _stale(want):
-        return LIB
+    the current sources (same source hash); return its path.  `stamps`:
+    the profiling build with the decode kernel's phase stamps, a separate
+    library."""
+    extra = STAMP_FLAGS if stamps else []
+    lib = LIB_STAMPS if stamps else LIB
+    want = source_hash(extra)
+    if not force and not verbose_ptxas and not _stale(want, lib):
+        return lib
     os.makedirs(LIBDIR, exist_ok=True)
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, f"-DABSP_BUILD_ID=\"{want}\"", "-shared",
+    tmp = lib + ".tmp"
+    cmd = [nvcc(), *ARCH, *FLAGS, *extra, f"-DABSP_BUILD_ID=\"{want}\"", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", INCLUDE, "-cudart", "static",
            "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES]
@@ -96,10 +103,10 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed building libabsp.so")
     if verbose_ptxas:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    with open(STAMP, "w") as f:
+    os.replace(tmp, lib)
+    with open(lib + ".build_id", "w") as f:
         f.write(want + "\n")
-    return LIB
+    return lib
 
 
 def main() -> None:

@@ -53,7 +53,28 @@
 
 namespace absp {
 
+#ifdef ABSP_PHASE_STAMPS
+// Phase stamps, compiled only into the separate profiling build: thread 0 of
+// CTAs 0..159 of a fused launch records globaltimer and clock64 at fixed
+// points (index k below), in 64 slots taken in launch order.
+__device__ unsigned long long g_stamp_t[64 * 160 * 24];
+__device__ long long g_stamp_c[64 * 160 * 24];
+int g_stamp_launches = 0;
+#endif
+
 namespace {
+
+#ifdef ABSP_PHASE_STAMPS
+__device__ __forceinline__ void stampk(int slot, int k) {
+    if (threadIdx.x == 0 && slot >= 0 && blockIdx.x < 160) {
+        const int i = (slot * 160 + blockIdx.x) * 24 + k;
+        g_stamp_t[i] = globaltimer_ns();
+        g_stamp_c[i] = clock64();
+    }
+}
+#else
+__device__ __forceinline__ void stampk(int, int) {}
+#endif
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -90,6 +111,7 @@ struct Params {
     uint32_t ring_off;            // code ring inside region B, past the select scratch
     uint32_t ptrow_off;           // staged page-table row, after the list
     int32_t pt_cap;               // entries the staged row holds (0: none)
+    int32_t stamp_slot;           // phase-stamp slot (profiling build), else -1
 };
 
 // per-head score weights for the group-max variant: [G][8 lanes][20]
@@ -321,7 +343,7 @@ __device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int
 // barrier.
 __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float mn, float mx,
                                            int32_t* out, int lo, int hi, uint32_t* scratch,
-                                           Small& sm) {
+                                           Small& sm, int stamp_slot) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (k >= n) {
         for (int i = max(0, lo) + tid; i < min(n, hi); i += kThreads) out[i - lo] = i;
@@ -373,6 +395,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
             }
         }
         __syncthreads();
+        stampk(stamp_slot, 11);                  // histogram done
         {
             // thread t owns bins 4(255-t) .. 4(255-t)+3 (one 16-byte load);
             // an exclusive scan in thread order counts the scores above them
@@ -396,6 +419,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
         }
         __syncthreads();
         const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
+        stampk(stamp_slot, 12);                  // boundary bin known
         if (m <= kMaxCand) {
             // one pass: a ballot word per 32 scores marks those above bin
             // bstar (selected); the scores inside bstar become candidates,
@@ -449,6 +473,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
             }
             if (lane == 0) sm.scan[warp] = cnt;
             __syncthreads();
+            stampk(stamp_slot, 13);              // ballot words and candidates out
             if (!all_in) {
                 // exact rank among the candidates: larger key first, ties to
                 // the lower index; the `need` best join the selection
@@ -484,6 +509,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                 }
                 __syncthreads();
             }
+            stampk(stamp_slot, 14);              // boundary candidates ranked
             block_extract_bitmap(inw, nwords, wpw, sm.scan, out, lo, hi);
             __syncthreads();
             return;
@@ -519,6 +545,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     int32_t* sel_s = reinterpret_cast<int32_t*>(base + p.qs_off + p.kv.G * kD * 2);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    stampk(p.stamp_slot, 0);                     // entry
     const uint32_t C = cluster_nctarank();
     const uint32_t rank = cluster_ctarank();
     // C (a power of two), bs and bs / 16 are powers of two: shifts, not
@@ -660,6 +687,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         pdl_wait();
         pdl_trigger();
     }
+    stampk(p.stamp_slot, 1);                     // released by the preceding launch
     int K = 0;
     int sel_lo = 0, sel_hi = 0;  // list entries held in sel_s
 
@@ -718,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             }
         }
         __syncthreads();
+        stampk(p.stamp_slot, 2);                 // query and weights ready
         const int sub = tid & 7, grp = tid >> 3;  // 32 groups of 8 lanes
         float wr[16], zr[16];
         float kz = 0.0f;  // this lane's share of sum_ch w[ch] * zp[ch], scaled
@@ -894,6 +923,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                 return make_float4(sc[0], sc[1], sc[2], sc[3]);
             });
         }
+        stampk(p.stamp_slot, 3);                 // own rows scored
         // this CTA's score range, sent along with the scores
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -919,6 +949,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         if (MODE == kModeSelect && rank != 0) return;
         // ------------------------------------- B: every score arrived --
         mbar_wait_bounded<true>(bar_score, 0, p.err, 4, kWaitNs);
+        stampk(p.stamp_slot, 4);                 // every CTA's scores here
 
         // --------------------------------------------------- C: select --
         float2 rv[16];                       // C <= 16: a tree, not a chain
@@ -946,7 +977,8 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             sel_hi = ppe > ppb ? ((ppe - 1) >> lgspb) + 1 : sel_lo;
         }
         block_topk(scores, n, K, smin, smax, sel_s, sel_lo, sel_hi,
-                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm);
+                   reinterpret_cast<uint32_t*>(regB + p.scratch_off), sm, p.stamp_slot);
+        stampk(p.stamp_slot, 5);                 // top-K done
         if (MODE == kModeSelect) {
             int32_t* dst = p.sel + (static_cast<int64_t>(s) * Hkv + h) * p.kmax;
             for (int i = tid; i < K; i += kThreads) dst[i] = sel_s[i];  // [0, K) held
@@ -1075,14 +1107,18 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
 
         // (the select, or the copy of a given selection, ended with a barrier:
         // no thread reads the scores in region B any more)
+        stampk(p.stamp_slot, 16);
         resolve(0);
+        stampk(p.stamp_slot, 17);                // page ids of the first 32 pages
         int vnext = cnt_w > 0 ? issue(0) : 0;
+        stampk(p.stamp_slot, 15);                // first page copies issued
 #pragma unroll 1
         for (int i = 1; i <= ABSP_PAGE_PREFETCH; ++i) prefetch(i);
 #pragma unroll 1
         for (int i = 0; i < cnt_w; ++i) {
             const int valid = vnext;
             mbar_wait_bounded(smem_u32(&sm.bar_page[warp]), i & 1, p.err, 2, kWaitNs);
+            if (i == 0) stampk(p.stamp_slot, 6);  // warp 0's first page landed
             if (valid > 0) {
                 uint8_t* pg = wbuf;
                 const uint32_t kb = smem_u32(pg), vb = kb + 4096;
@@ -1196,6 +1232,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             }
             if (ABSP_PAGE_PREFETCH > 0) prefetch(i + 1 + ABSP_PAGE_PREFETCH);
         }
+        stampk(p.stamp_slot, 7);                 // warp 0 attended its pages
         l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
         l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
         l8 += __shfl_xor_sync(0xffffffffu, l8, 1);
@@ -1238,6 +1275,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             }
         }
         __syncthreads();
+        stampk(p.stamp_slot, 8);                 // warp partials in shared memory
         if constexpr ((MODE & kModeSelect) == 0) cluster_wait();  // B0
         __nv_bfloat16* outp = p.out + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD;
         // this CTA's partial of 4 channels of one row, with the row's M and
@@ -1312,6 +1350,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         // after its own page lookups, so no CTA leaves while another may
         // still read its staged page ids)
         mbar_wait_bounded<true>(bar_merge, 0, p.err, 3, kWaitNs);
+        stampk(p.stamp_slot, 9);                 // every CTA's partial slice here
         __syncthreads();                                    // this CTA's own stores
         // per (row, partial) weight exp2(M_r - M) / L: one thread per pair
         // (G * C <= 256), the C partials of a row on C consecutive lanes
@@ -1364,6 +1403,10 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             if (act && qtr == 0)
                 *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) = pack_bf16x2(a0, a1);
         }
+#ifdef ABSP_PHASE_STAMPS
+        __syncthreads();
+#endif
+        stampk(p.stamp_slot, 10);                // output slice written
     }
 }
 
@@ -1519,6 +1562,11 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     prm.err = a.err;
     prm.qk_scale_log2 = kLog2e / sqrtf(static_cast<float>(kD));
     prm.wg_off = 0;
+#ifdef ABSP_PHASE_STAMPS
+    prm.stamp_slot = mode == kModeFull ? (g_stamp_launches++ & 63) : -1;
+#else
+    prm.stamp_slot = -1;
+#endif
 
     int C = pick_cluster(pairs, num_sms);
     cudaError_t e = cudaSuccess;
@@ -1612,3 +1660,16 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
 }
 
 }  // namespace absp
+
+#ifdef ABSP_PHASE_STAMPS
+// Profiling build only: restart the slot count; copy the stamps (globaltimer
+// ns, then clock64 ticks, each [64][160][24]) to host memory.
+extern "C" __attribute__((visibility("default"))) void absp_phase_stamps_reset() {
+    absp::g_stamp_launches = 0;
+}
+extern "C" __attribute__((visibility("default"))) int absp_phase_stamps_copy(void* t, void* c) {
+    cudaError_t e = cudaMemcpyFromSymbol(t, absp::g_stamp_t, sizeof(absp::g_stamp_t));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(c, absp::g_stamp_c, sizeof(absp::g_stamp_c));
+    return static_cast<int>(e);
+}
+#endif
