@@ -1508,11 +1508,30 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
 #define ABSP_DECODE_CTAS_PER_SM 2   // CTA count the cluster size aims for, per SM
 #endif
 
+#ifndef ABSP_DECODE_ROWS_PER_CTA
+#define ABSP_DECODE_ROWS_PER_CTA 256  // score rows per CTA the cluster size aims for
+#endif
+#ifndef ABSP_DECODE_PAGES_PER_CTA
+#define ABSP_DECODE_PAGES_PER_CTA 16  // selected pages per CTA (two per warp)
+#endif
+
 // Cluster size: enough CTAs to cover the SMs about ABSP_DECODE_CTAS_PER_SM
-// times, at most 16.
-static int pick_cluster(int pairs, int num_sms) {
+// times, at most 16, and no more than it takes to give each CTA about
+// ABSP_DECODE_ROWS_PER_CTA of the largest head's score rows (nmax blocks)
+// and about ABSP_DECODE_PAGES_PER_CTA of a head's selected pages (budget /
+// 16).  Past that point more CTAs per head add cluster-wide waits and
+// merge partials but take little work off the chain: measured on the
+// Llama-shaped 32K layers (up to 2048 blocks, 128 selected pages per head),
+// 8 CTAs per head beat 16 at batch 1 (10.36 vs 10.46 us per layer-step) and
+// halve the time per launch of independent launches that overlap (3.5 vs
+// 6.9 us), while 4 CTAs (four pages per warp) took 13.7 us; on the 128K
+// layer (8192 blocks, 256 pages) 16 beat 8 (18.0 vs 19.6 us).
+static int pick_cluster(int pairs, int num_sms, int nmax, int budget) {
+    const int need = std::max((nmax + ABSP_DECODE_ROWS_PER_CTA - 1) / ABSP_DECODE_ROWS_PER_CTA,
+                              (budget / kPage + ABSP_DECODE_PAGES_PER_CTA - 1) /
+                                  ABSP_DECODE_PAGES_PER_CTA);
     int C = 1;
-    while (C < 16 && pairs * C * 2 <= ABSP_DECODE_CTAS_PER_SM * num_sms) C *= 2;
+    while (C < 16 && pairs * C * 2 <= ABSP_DECODE_CTAS_PER_SM * num_sms && C < need) C *= 2;
     return C;
 }
 
@@ -1568,7 +1587,7 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     prm.stamp_slot = -1;
 #endif
 
-    int C = pick_cluster(pairs, num_sms);
+    int C = pick_cluster(pairs, num_sms, a.nmax, a.budget);
     cudaError_t e = cudaSuccess;
     for (; C >= 1; C /= 2) {
         // region B: scores + select scratch + the code ring, then this CTA's
