@@ -28,6 +28,7 @@ ABSP_ERR_TIMEOUT = 5
 
 ABSP_STEP_EARLY_PREFETCH = 1
 ABSP_STEP_GROUP_MAX = 2
+ABSP_STEP_THROUGHPUT = 4
 ABSP_STEP_DIAG_WAIT_TIMEOUT = 0x100
 ABSP_CENTROIDS_INT4 = 0
 ABSP_CENTROIDS_BF16 = 1

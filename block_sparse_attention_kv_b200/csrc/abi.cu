@@ -217,6 +217,7 @@ absp_status run_decode(int mode, const absp_layer_kv* kv, const absp_centroids* 
     a.cfmt = cent ? cent->format : ABSP_CENTROIDS_INT4;
     a.group_max = (flags & ABSP_STEP_GROUP_MAX) != 0 ? 1 : 0;
     a.diag_timeout = (flags & ABSP_STEP_DIAG_WAIT_TIMEOUT) != 0 ? 1 : 0;
+    a.throughput = (flags & ABSP_STEP_THROUGHPUT) != 0 ? 1 : 0;
     if (a.diag_timeout && (mode == kModeAttend || a.group_max || a.cfmt != ABSP_CENTROIDS_INT4 ||
                            d.G > 8 || (flags & ABSP_STEP_EARLY_PREFETCH) != 0))
         return ABSP_ERR_UNSUPPORTED;
@@ -399,7 +400,7 @@ absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* c
                                 size_t ws_bytes, uint32_t flags, void* stream) {
     ABSP_TRACE("absp_decode_step_ex");
     if ((flags & ~static_cast<uint32_t>(ABSP_STEP_EARLY_PREFETCH | ABSP_STEP_GROUP_MAX |
-                                        ABSP_STEP_DIAG_WAIT_TIMEOUT)) != 0)
+                                        ABSP_STEP_THROUGHPUT | ABSP_STEP_DIAG_WAIT_TIMEOUT)) != 0)
         return ABSP_ERR_INVALID_ARG;
     return run_decode(kModeFull, kv, cent, q, budget_tokens, nullptr, nullptr, out, ws, ws_bytes,
                       stream, flags);

@@ -360,6 +360,7 @@ struct DecodeArgs {
     int32_t cfmt;                 // centroid format (ABSP_CENTROIDS_*)
     int32_t group_max;            // score = max over the GQA group's heads
     int32_t diag_timeout;         // ABSP_STEP_DIAG_WAIT_TIMEOUT: the failure-path diagnostic
+    int32_t throughput;           // ABSP_STEP_THROUGHPUT: half as many CTAs per head
 };
 // early_prefetch: codes, parameters, lengths and page table are read before
 // the programmatic-dependency wait (only the query after it).

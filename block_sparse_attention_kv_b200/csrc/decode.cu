@@ -1526,10 +1526,11 @@ cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool p
 // halve the time per launch of independent launches that overlap (3.5 vs
 // 6.9 us), while 4 CTAs (four pages per warp) took 13.7 us; on the 128K
 // layer (8192 blocks, 256 pages) 16 beat 8 (18.0 vs 19.6 us).
-static int pick_cluster(int pairs, int num_sms, int nmax, int budget) {
-    const int need = std::max((nmax + ABSP_DECODE_ROWS_PER_CTA - 1) / ABSP_DECODE_ROWS_PER_CTA,
-                              (budget / kPage + ABSP_DECODE_PAGES_PER_CTA - 1) /
-                                  ABSP_DECODE_PAGES_PER_CTA);
+// With the throughput hint the work per CTA doubles (half the CTAs).
+static int pick_cluster(int pairs, int num_sms, int nmax, int budget, bool throughput) {
+    const int rows = ABSP_DECODE_ROWS_PER_CTA << (throughput ? 1 : 0);
+    const int pages = ABSP_DECODE_PAGES_PER_CTA << (throughput ? 1 : 0);
+    const int need = std::max((nmax + rows - 1) / rows, (budget / kPage + pages - 1) / pages);
     int C = 1;
     while (C < 16 && pairs * C * 2 <= ABSP_DECODE_CTAS_PER_SM * num_sms && C < need) C *= 2;
     return C;
@@ -1587,7 +1588,7 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
     prm.stamp_slot = -1;
 #endif
 
-    int C = pick_cluster(pairs, num_sms, a.nmax, a.budget);
+    int C = pick_cluster(pairs, num_sms, a.nmax, a.budget, a.throughput != 0);
     cudaError_t e = cudaSuccess;
     for (; C >= 1; C /= 2) {
         // region B: scores + select scratch + the code ring, then this CTA's

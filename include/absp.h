@@ -272,11 +272,19 @@ ABSP_API absp_status absp_decode_step(const absp_layer_kv* kv, const absp_centro
  * group of at most 8 and without ABSP_STEP_EARLY_PREFETCH
  * (ABSP_ERR_UNSUPPORTED otherwise). */
 #define ABSP_STEP_DIAG_WAIT_TIMEOUT 0x100u
+/* ABSP_STEP_THROUGHPUT: a hint that the caller overlaps this launch with
+ * other independent launches (separate requests on several streams, no
+ * dependency between them).  Each (seq, kv_head) then gets half as many
+ * CTAs, each doing twice the work, so that more launches are resident at
+ * once: longer per launch, more launches per second in aggregate.  The
+ * selection is the same; the output differs from the default only in the
+ * order of the softmax merge's partial sums (fp32 rounding). */
+#define ABSP_STEP_THROUGHPUT 0x4u
 
 /* absp_decode_step with flags (ABSP_STEP_EARLY_PREFETCH, ABSP_STEP_GROUP_MAX,
- * ABSP_STEP_DIAG_WAIT_TIMEOUT; other bits are rejected).  Without
- * ABSP_STEP_GROUP_MAX and the diagnostic, same results as
- * absp_decode_step. */
+ * ABSP_STEP_THROUGHPUT, ABSP_STEP_DIAG_WAIT_TIMEOUT; other bits are
+ * rejected).  Without ABSP_STEP_GROUP_MAX, ABSP_STEP_THROUGHPUT and the
+ * diagnostic, same results as absp_decode_step. */
 ABSP_API absp_status absp_decode_step_ex(const absp_layer_kv* kv, const absp_centroids* cent,
                                          const void* q, int32_t budget_tokens, void* out,
                                          void* ws, size_t ws_bytes, uint32_t flags,

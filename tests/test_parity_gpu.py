@@ -238,6 +238,26 @@ def test_group_max_llama31_8b_32k(lib):
     run_case(lib, synth.WORKLOADS["llama31_8b_32k"], flags=abi.ABSP_STEP_GROUP_MAX)
 
 
+@pytest.mark.parametrize("wname", ["tiny_8k", "llama31_8b_32k"])
+def test_throughput_hint_matches_the_oracle(lib, wname):
+    # ABSP_STEP_THROUGHPUT halves the CTAs per head: the same selection, the
+    # output equal up to the merge order's rounding, so within the oracle
+    # tolerance and bf16-close to the default step's
+    abi, pipeline = lib
+    rep, dl, res = run_case(lib, synth.WORKLOADS[wname])
+    want = dl.out.clone()
+    dl.out.zero_()
+    dl.decode_step(flags=abi.ABSP_STEP_THROUGHPUT | abi.ABSP_STEP_EARLY_PREFETCH)
+    dl.check()
+    torch.cuda.synchronize()
+    got = dl.out.float().cpu().numpy()
+    rep2 = PR.Report()
+    PR.compare_outputs(rep2, got, res.out)
+    assert rep2.ok(), rep2.notes[:10]
+    diff = (dl.out.float() - want.float()).abs().max().item()
+    assert diff <= 2e-2 * max(1.0, want.float().abs().max().item()), diff
+
+
 def test_host_buffers_match_device_step(lib):
     abi, pipeline = lib
     w = synth.custom("host_io", 2, 8, 2, [3000, 900], [16, 64], 512, seed=40)
