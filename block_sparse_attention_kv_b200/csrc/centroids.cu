@@ -62,16 +62,22 @@ __device__ __forceinline__ double mean_of(double x, int cnt, double inv_pow2) {
     return (cnt & (cnt - 1)) == 0 ? x * inv_pow2 : x / static_cast<double>(cnt);
 }
 
-// rint(c / sc) (IEEE division, round half to even) without dividing on the
-// common path: r = c * inv (inv = 1 / sc rounded) is within 2^-51 |c/sc| of
-// the quotient, so unless r lies within 2^-48 max(|r|, 1) of a half-integer
-// (where rint could jump) its rint is the quotient's; otherwise divide.
-__device__ __forceinline__ double rint_div(double c, double sc, double inv) {
+// The INT4 code clamp(rint(c / sc) + zp, 0, 15) (IEEE division, round half
+// to even, fp64) without dividing on the common path: r = c * inv (inv =
+// 1 / sc rounded) and the rounded quotient are both within about 2^-52 |r|
+// of c / sc, under 2^-31 for |r| < 2^20, so when r lies at least 2^-28 from
+// every half-integer (|r - rint(r)| <= 0.5 - 2^-28) both round to the same
+// integer; the offset and clamp then run on integers.  Larger quotients and
+// residues nearer 0.5 take the exact path.
+__device__ __forceinline__ uint32_t int4_code(double c, double sc, double inv, int32_t zp) {
     const double r = c * inv;
-    const double fl = floor(r);
-    const double d = r - fl;
-    if (fabs(d - 0.5) <= fmax(fabs(r), 1.0) * 0x1p-48) return rint(c / sc);
-    return d > 0.5 ? fl + 1.0 : fl;
+    const double fl = rint(r);
+    if (fabs(r) < 0x1p20 && fabs(r - fl) <= 0.5 - 0x1p-28) {
+        const long long v = static_cast<long long>(fl) + zp;
+        return static_cast<uint32_t>(v < 0 ? 0 : v > 15 ? 15 : v);
+    }
+    const double qv = fmin(fmax(rint(c / sc) + static_cast<double>(zp), 0.0), 15.0);
+    return static_cast<uint32_t>(qv);
 }
 
 // ---------------------------------------------------------------------------
@@ -397,11 +403,12 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
         }
     }
     __syncthreads();
-    double sc[4], zz[4], iv[4];
+    double sc[4], iv[4];
+    int32_t zi[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         sc[i] = s_par[0][lane * 4 + i];
-        zz[i] = s_par[1][lane * 4 + i];
+        zi[i] = static_cast<int32_t>(s_par[1][lane * 4 + i]);   // an int32 held exactly
         iv[i] = s_par[2][lane * 4 + i];
     }
     auto code_rows = [&](int b0, const double (&cb)[kRows][4]) {
@@ -412,12 +419,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
             uint32_t packed = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t code = 0;
-                if (sc[i] != 0.0) {
-                    double qv = rint_div(cb[q][i], sc[i], iv[i]) + zz[i];
-                    qv = fmin(fmax(qv, 0.0), 15.0);
-                    code = static_cast<uint32_t>(qv);
-                }
+                const uint32_t code = sc[i] != 0.0 ? int4_code(cb[q][i], sc[i], iv[i], zi[i]) : 0u;
                 packed |= code << (4 * i);
             }
             *reinterpret_cast<uint16_t*>(codes + (row0 + b) * kRowBytes + lane * 2) =
