@@ -315,10 +315,44 @@ __device__ __noinline__ void compact_by_threshold(const float* sc, int n, uint32
 }
 
 // Entries [lo, hi) of the ascending list of the set bits of
+// Long runs of block_extract_bitmap (more than 8 words per warp, over 2048
+// scores), kept out of line so that the short path's code is unchanged:
+// lane l takes word 32 g + l of the warp's run (g = 0, 1, ...), a prefix
+// sum of the words' bit counts over the lanes gives each word's first
+// position, and the lane writes the word's set bits in order, those within
+// [lo, hi).  `pos`: the set bits of the warps before.
+__device__ __noinline__ void extract_bitmap_long(const uint32_t* bitmap, int j0, int j1,
+                                                 uint32_t pos, int32_t* out, int lo, int hi) {
+    const int lane = threadIdx.x & 31;
+    for (int jb = j0; jb < j1 && static_cast<int>(pos) < hi; jb += 32) {
+        const int j = jb + lane;
+        const uint32_t bits = j < j1 ? bitmap[j] : 0u;
+        const uint32_t c = __popc(bits);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int at = static_cast<int>(pos + incl - c);
+        if (at < hi && at + static_cast<int>(c) > lo) {
+            uint32_t b = bits;
+            while (b != 0u) {
+                const int bit = __ffs(b) - 1;
+                b &= b - 1u;
+                if (at >= lo && at < hi) out[at - lo] = j * 32 + bit;
+                ++at;
+            }
+        }
+        pos += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
 // bitmap[0..nwords), by the whole block: warp w owns the contiguous words
 // [w * wpw, (w + 1) * wpw) and wcnt[w] holds the number of set bits in them.
 // Each lane places its own bit of every word: position = the set bits of the
-// warps before, of the words before in its run, and of the lanes below.
+// warps before, of the words before in its run, and of the lanes below
+// (runs of more than 8 words: extract_bitmap_long).
 __device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int nwords, int wpw,
                                                      const uint32_t* wcnt, int32_t* out, int lo,
                                                      int hi) {
@@ -326,8 +360,12 @@ __device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int
     uint32_t pos = 0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) pos += w < warp ? wcnt[w] : 0u;
-    const uint32_t lt = (1u << lane) - 1u;
     const int j0 = min(nwords, warp * wpw), j1 = min(nwords, j0 + wpw);
+    if (wpw > 8) {
+        extract_bitmap_long(bitmap, j0, j1, pos, out, lo, hi);
+        return;
+    }
+    const uint32_t lt = (1u << lane) - 1u;
     for (int j = j0; j < j1 && static_cast<int>(pos) < hi; ++j) {
         const uint32_t bits = bitmap[j];
         const int at = static_cast<int>(pos + __popc(bits & lt));
