@@ -112,6 +112,7 @@ struct Params {
     uint32_t ptrow_off;           // staged page-table row, after the list
     int32_t pt_cap;               // entries the staged row holds (0: none)
     int32_t stamp_slot;           // phase-stamp slot (profiling build), else -1
+    int32_t npbuf;                // page buffers per warp (1, or 2 when one CTA per SM is enough)
 };
 
 // per-head score weights for the group-max variant: [G][8 lanes][20]
@@ -123,7 +124,7 @@ constexpr int kPtStage = 512;    // page-table entries a CTA stages for its own 
 struct Small {                    // fixed-size shared scratch
     int32_t pt[kPtStage];         // page ids of the pages of this CTA's scored rows
     unsigned long long bar_code[kMaxStages];
-    unsigned long long bar_page[kWarps];
+    unsigned long long bar_page[2 * kWarps];   // [warp][page buffer]
     unsigned long long bar_merge;
     unsigned long long bar_score;
     float2 cmm[16];               // (min, max) of each cluster CTA's scores
@@ -568,7 +569,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 // score barrier expects 16 bytes that are never sent and every bounded wait
 // gives up after 1 ms, so the score wait runs out, records ABSP_ERR_TIMEOUT
 // and the kernel carries on to its normal end.
-template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM, bool DIAG>
+template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM, bool DIAG, int NPB>
 __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
@@ -613,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
     }
     if (tid == 0) {
         for (int i = 0; i < kMaxStages; ++i) mbar_init(smem_u32(&sm.bar_code[i]), 1);
-        for (int w = 0; w < kWarps; ++w) mbar_init(smem_u32(&sm.bar_page[w]), 1);
+        for (int w = 0; w < 2 * kWarps; ++w) mbar_init(smem_u32(&sm.bar_page[w]), 1);
         mbar_init(smem_u32(&sm.bar_score), 1);
         mbar_init(smem_u32(&sm.bar_merge), 1);
         fence_mbar_init();
@@ -1065,7 +1066,9 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         float m0 = -FLT_MAX, m8 = -FLT_MAX, l0 = 0.0f, l8 = 0.0f;
         bool any0 = false;  // this warp has seen at least one valid token
         const float qks = p.qk_scale_log2;
-        uint8_t* wbuf = regB + warp * kPageSmem;  // this warp's page buffer
+        // this warp's page buffers: page i goes to buffer i % NPB
+        constexpr int npbuf = NPB;
+        uint8_t* wbuf = regB + warp * npbuf * kPageSmem;
 
         // Pages of this warp, 32 at a time: lane l resolves page c0 + l into
         // its physical page id and valid token count (one parallel round of
@@ -1116,12 +1119,13 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
             const int valid = __shfl_sync(0xffffffffu, my_valid, i & 31);
             const int phys = __shfl_sync(0xffffffffu, my_phys, i & 31);
             if (lane == 0) {
-                const uint32_t bar = smem_u32(&sm.bar_page[warp]);
+                const int k = i & (npbuf - 1);
+                const uint32_t bar = smem_u32(&sm.bar_page[2 * warp + k]);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, valid > 0 ? kPageSmem : 0);
                 if (valid > 0) {
                     const int y = (phys * Hkv + h) * kPage;
-                    const uint32_t dst = smem_u32(wbuf);
+                    const uint32_t dst = smem_u32(wbuf + k * kPageSmem);
                     tma_load_2d(dst, &tmk, 0, y, bar);
                     tma_load_2d(dst + 2048, &tmk, 64, y, bar);
                     tma_load_2d(dst + 4096, &tmv, 0, y, bar);
@@ -1148,17 +1152,21 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
         stampk(p.stamp_slot, 16);
         resolve(0);
         stampk(p.stamp_slot, 17);                // page ids of the first 32 pages
-        int vnext = cnt_w > 0 ? issue(0) : 0;
+        // the valid token counts of the pages in flight, by buffer
+        int vbuf0 = cnt_w > 0 ? issue(0) : 0;
+        int vbuf1 = npbuf == 2 && cnt_w > 1 ? issue(1) : 0;
         stampk(p.stamp_slot, 15);                // first page copies issued
 #pragma unroll 1
         for (int i = 1; i <= ABSP_PAGE_PREFETCH; ++i) prefetch(i);
 #pragma unroll 1
         for (int i = 0; i < cnt_w; ++i) {
-            const int valid = vnext;
-            mbar_wait_bounded(smem_u32(&sm.bar_page[warp]), i & 1, p.err, 2, kWaitNs);
+            const int k = i & (npbuf - 1);
+            const int valid = k ? vbuf1 : vbuf0;
+            mbar_wait_bounded(smem_u32(&sm.bar_page[2 * warp + k]), (i >> (npbuf - 1)) & 1, p.err,
+                              2, kWaitNs);
             if (i == 0) stampk(p.stamp_slot, 6);  // warp 0's first page landed
             if (valid > 0) {
-                uint8_t* pg = wbuf;
+                uint8_t* pg = wbuf + k * kPageSmem;
                 const uint32_t kb = smem_u32(pg), vb = kb + 4096;
                 if (valid < kPage) {
                     // zero the V rows past the sequence end (they may hold
@@ -1263,10 +1271,11 @@ __global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
                     }
                 }
             }
-            if (i + 1 < cnt_w) {
+            if (i + npbuf < cnt_w) {
                 fence_proxy_async_smem();  // this lane's reads/writes of the buffer
                 __syncwarp();              // before its next tensor copy
-                vnext = issue(i + 1);
+                const int v = issue(i + npbuf);
+                if (k) vbuf1 = v; else vbuf0 = v;
             }
             if (ABSP_PAGE_PREFETCH > 0) prefetch(i + 1 + ABSP_PAGE_PREFETCH);
         }
@@ -1469,11 +1478,11 @@ struct ShapeCache {
     }
 };
 
-template <int MODE, bool BIG, bool EARLY, bool BF16C, bool GM, bool DIAG = false>
+template <int MODE, bool BIG, bool EARLY, bool BF16C, bool GM, bool DIAG = false, int NPB = 1>
 cudaError_t launch_mode(const Params& prm, size_t smem, int C, int pairs, bool pdl,
                         const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st,
                         bool* fits) {
-    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C, GM, DIAG>;
+    auto kern = decode_kernel<MODE, BIG, EARLY, BF16C, GM, DIAG, NPB>;
     // per device (function attributes belong to a device's context) and
     // per shape: whether one cluster of C CTAs with `smem` bytes fits
     static std::mutex mu;
@@ -1642,11 +1651,22 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
             ring = (used + 127) & ~static_cast<size_t>(127);
             regB = std::max(regB, ring + static_cast<size_t>(kStages) * kStageBytes);
         }
+        // Page buffers per warp: a second one overlaps a page's copy with the
+        // previous page's attention but takes the shared memory of a second
+        // CTA per SM.  The default fused step (INT4, sum, GQA <= 8, no
+        // throughput hint) has its own kernel instance with two, used when
+        // the launch's CTAs fit on half the SMs, so that one CTA per SM
+        // still leaves room for the next launch; every other instance keeps
+        // one (measured: the batch-1 Llama-shaped layer-step 10.37 -> 10.12
+        // us; with the extra buffer logic in every instance the batched
+        // workloads lost 1 %).
+        prm.npbuf = mode == kModeFull && !big && a.cfmt != ABSP_CENTROIDS_BF16 &&
+                            !a.group_max && !a.diag_timeout && !a.throughput &&
+                            pairs * C * 2 <= num_sms
+                        ? 2
+                        : 1;
         if (do_attend) {
-            // one page buffer per warp: a second one (double buffering)
-            // halves the resident CTAs per SM and was slower on every
-            // workload measured
-            regB = std::max(regB, static_cast<size_t>(kWarps) * kPageSmem);
+            regB = std::max(regB, static_cast<size_t>(kWarps) * prm.npbuf * kPageSmem);
             regB = std::max(regB, static_cast<size_t>(kWarps) * G * (kD + 2) * 4);
             // the slice merge's receive buffers: C partial slices of G x
             // 128/C channels and (M, L) per row
@@ -1672,10 +1692,10 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
                              static_cast<size_t>(a.kmax) * 4 + 15) & ~static_cast<size_t>(15);
         prm.ptrow_off = static_cast<uint32_t>(tail);
         prm.pt_cap = 0;
-        constexpr size_t kTwoPerSm = 112 * 1024;
-        if (do_select && do_attend && 1024 + tail < kTwoPerSm)
+        const size_t share = prm.npbuf == 2 ? 224 * 1024 : 112 * 1024;  // per-CTA budget
+        if (do_select && do_attend && 1024 + tail < share)
             prm.pt_cap = static_cast<int32_t>(
-                std::min<size_t>(a.kv.max_pages, (kTwoPerSm - 1024 - tail) / 4) & ~static_cast<size_t>(3));
+                std::min<size_t>(a.kv.max_pages, (share - 1024 - tail) / 4) & ~static_cast<size_t>(3));
         const size_t smem = 1024 + tail + static_cast<size_t>(prm.pt_cap) * 4;
         if (smem > 227 * 1024) return cudaErrorInvalidValue;
         bool fits = false;
@@ -1704,6 +1724,11 @@ cudaError_t launch_decode(int mode, const DecodeArgs& a, const CUtensorMap* tmk,
                                                               tmk, tmv, st, &fits)
                       : launch_variant<kModeFull, true, false>(bf, gm, prm, smem, C, pairs, pdl,
                                                                tmk, tmv, st, &fits);
+        } else if (prm.npbuf == 2) {
+            e = early ? launch_mode<kModeFull, false, true, false, false, false, 2>(
+                            prm, smem, C, pairs, pdl, tmk, tmv, st, &fits)
+                      : launch_mode<kModeFull, false, false, false, false, false, 2>(
+                            prm, smem, C, pairs, pdl, tmk, tmv, st, &fits);
         } else {
             e = early ? launch_variant<kModeFull, false, true>(bf, gm, prm, smem, C, pairs, pdl,
                                                                tmk, tmv, st, &fits)
