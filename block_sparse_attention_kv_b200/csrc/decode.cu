@@ -570,7 +570,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
 // gives up after 1 ms, so the score wait runs out, records ABSP_ERR_TIMEOUT
 // and the kernel carries on to its normal end.
 template <int MODE, bool BIG_GROUP, bool EARLY, bool BF16C, bool GM, bool DIAG, int NPB>
-__global__ void __launch_bounds__(kThreads, ABSP_DECODE_MIN_BLOCKS)
+__global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t smem_raw[];
