@@ -1113,7 +1113,9 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         };
 
         // page i of this warp: tensor copies of its K and V slices (every
-        // lane calls this; lane 0 issues)
+        // lane calls this; lane 0 issues).  The caller has ordered this
+        // lane's earlier generic accesses of the buffer before the copy
+        // (fence.proxy.async after the warp's last use of it).
         auto issue = [&](int i) -> int {
             if (i >= c0 + 32) resolve(i);
             const int valid = __shfl_sync(0xffffffffu, my_valid, i & 31);
@@ -1121,7 +1123,6 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
             if (lane == 0) {
                 const int k = i & (npbuf - 1);
                 const uint32_t bar = smem_u32(&sm.bar_page[2 * warp + k]);
-                fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, valid > 0 ? kPageSmem : 0);
                 if (valid > 0) {
                     const int y = (phys * Hkv + h) * kPage;
@@ -1152,7 +1153,12 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         stampk(p.stamp_slot, 16);
         resolve(0);
         stampk(p.stamp_slot, 17);                // page ids of the first 32 pages
-        // the valid token counts of the pages in flight, by buffer
+        // the valid token counts of the pages in flight, by buffer (the
+        // buffers held scores and select scratch before the barrier that
+        // ended the select: one proxy fence orders those accesses before
+        // the first copies)
+        fence_proxy_async_smem();
+        __syncwarp();
         int vbuf0 = cnt_w > 0 ? issue(0) : 0;
         int vbuf1 = npbuf == 2 && cnt_w > 1 ? issue(1) : 0;
         stampk(p.stamp_slot, 15);                // first page copies issued
