@@ -3,15 +3,15 @@
 // vectors of a head, once) and their INT4 asymmetric per-channel codes
 // (Fig. 8).
 //
-// Kernel shapes.  Both kernels tile a layer by (1024-token chunk, KV head,
+// Kernel shapes.  The build tiles a layer by (1024-token chunk, KV head,
 // sequence): every CTA covers the same number of tokens whatever the head's
 // block size (64, 32 or 16 blocks), so work is balanced across heads.
-//   build:    one warp per block; lane L owns channels 4L..4L+3 and reads
-//             8 bytes of every key row (a warp reads a full 256-byte row per
-//             instruction, coalesced).  Sums are fp64 in token order, so the
-//             result is bit-identical to a sequential fp64 mean.  The CTA
-//             reduces its per-channel min / max in shared memory and issues
-//             one atomic per channel (order-mapped fp64 keys).
+//   build:    one half-warp per block; lane l owns channels 8l..8l+7 and
+//             reads 16 bytes of every key row (a half-warp reads a whole
+//             256-byte row per instruction).  The sums equal the token-order
+//             fp64 sums bit for bit (block_sums).  The CTA reduces its
+//             per-channel min / max in shared memory and issues one atomic
+//             per channel (order-mapped fp64 keys).
 //   quantize: reads the fp64 centroids back, derives scale / zero point from
 //             the min / max (fp64, IEEE division, rint half-to-even) and
 //             writes packed nibbles: lane L writes 2 bytes of each 64-byte
@@ -78,6 +78,30 @@ __device__ __forceinline__ uint32_t int4_code(double c, double sc, double inv, i
     }
     const double qv = fmin(fmax(rint(c / sc) + static_cast<double>(zp), 0.0), 15.0);
     return static_cast<uint32_t>(qv);
+}
+
+// INT4 parameters of one channel from its order-mapped min key and the key
+// of its negated max (Fig. 8): scf = fp32((max - min) / 15) and, in fp64,
+// sc = scf and zi = rint(-min / sc) saturated to int32; a channel with
+// max == min, or a (sequence, head) with no rows (any = false), gets 0 / 0.
+__device__ __forceinline__ void channel_params(unsigned long long kmn, unsigned long long knmx,
+                                               bool any, float& scf, double& sc, int32_t& zi) {
+    scf = 0.0f;
+    sc = 0.0;
+    zi = 0;
+    if (!any) return;
+    const double mn = unord_f64(kmn);
+    const double mx = -unord_f64(knmx);
+    if (mx > mn) {
+        const float f = __double2float_rn((mx - mn) / 15.0);
+        if (f > 0.0f) {
+            scf = f;
+            sc = static_cast<double>(f);
+            double zr = rint(-mn / sc);
+            zr = fmin(fmax(zr, -2147483648.0), 2147483647.0);
+            zi = static_cast<int32_t>(zr);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -375,27 +399,14 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
     if (threadIdx.x < kD) {
         const int d = threadIdx.x;
         const int64_t pi = (static_cast<int64_t>(s) * kv.Hkv + h) * kD + d;
-        double sc = 0.0, z = 0.0;
-        float scf = 0.0f;
-        int32_t zi = 0;
-        if (n > 0) {
-            const int64_t pairs = static_cast<int64_t>(kv.S) * kv.Hkv * kD;
-            const double mn = unord_f64(w.minmax[pi]);
-            const double mx = -unord_f64(w.minmax[pairs + pi]);
-            if (mx > mn) {
-                const float f = __double2float_rn((mx - mn) / 15.0);
-                if (f > 0.0f) {
-                    scf = f;
-                    sc = static_cast<double>(f);
-                    double zr = rint(-mn / sc);
-                    zr = fmin(fmax(zr, -2147483648.0), 2147483647.0);
-                    zi = static_cast<int32_t>(zr);
-                    z = static_cast<double>(zi);
-                }
-            }
-        }
+        const int64_t pairs = static_cast<int64_t>(kv.S) * kv.Hkv * kD;
+        float scf;
+        double sc;
+        int32_t zi;
+        channel_params(n > 0 ? w.minmax[pi] : 0ull, n > 0 ? w.minmax[pairs + pi] : 0ull, n > 0,
+                       scf, sc, zi);
         s_par[0][d] = sc;
-        s_par[1][d] = z;
+        s_par[1][d] = static_cast<double>(zi);
         s_par[2][d] = sc != 0.0 ? 1.0 / sc : 0.0;
         if (grp == 0) {
             scale_out[pi] = scf;

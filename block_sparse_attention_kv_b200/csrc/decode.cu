@@ -433,6 +433,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                 }
             }
         }
+        stampk(stamp_slot, 21);                  // warp 0's histogram updates issued
         __syncthreads();
         stampk(stamp_slot, 11);                  // histogram done
         {
@@ -511,6 +512,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                 }
             }
             if (lane == 0) sm.scan[warp] = cnt;
+            stampk(stamp_slot, 22);              // warp 0's ballot words out
             __syncthreads();
             stampk(stamp_slot, 13);              // ballot words and candidates out
             if (!all_in) {
@@ -694,6 +696,12 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
                                  static_cast<uint32_t>(min(kSRows, nrows - c * kSRows) * kRow));
         }
     }
+    if constexpr (kSelect) {
+        // the select's histogram bins (in region B's select scratch, which
+        // nothing touches before the select), zeroed ahead of the wait
+        uint32_t* hist = reinterpret_cast<uint32_t*>(regB + p.scratch_off);
+        for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+    }
     // B0 arrive (release: the barrier set-up above is visible cluster-wide
     // once B0 completes); matched by the wait before the first remote access.
     cluster_arrive();
@@ -811,10 +819,7 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         const uint32_t bar_score = smem_u32(&sm.bar_score);
         float lmin = INFINITY, lmax = -INFINITY;
         if constexpr (!EARLY) cluster_wait();  // B0: every CTA of the cluster is running
-        {   // histogram bins of the select, zeroed while the codes stream in
-            uint32_t* hist = reinterpret_cast<uint32_t*>(regB + p.scratch_off);
-            for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
-        }
+        stampk(p.stamp_slot, 18);                // scoring starts
         // The chunk loop over the code ring; score4(sbuf, r4, rows) gives one
         // 8-lane group's scores of rows r4 .. r4 + 3 of a stage (values for
         // rows past `rows` are discarded here).
@@ -823,6 +828,7 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
             for (int c = 0; c < nchunks; ++c) {
                 const int stage = c % NS;
                 mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / NS) & 1, p.err, 1, kWaitNs);
+                if (c == 0) stampk(p.stamp_slot, 19);  // first code stage here
                 const int rows = min(kSRows, nrows - c * kSRows);
                 const uint8_t* sbuf = stage_buf(stage);
 #pragma unroll 1
@@ -853,6 +859,7 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
                         }
                     }
                 }
+                if (c == 0) stampk(p.stamp_slot, 20);  // warp 0 scored the first stage
                 __syncthreads();
                 if (tid == 0 && c + NS < nchunks) {
                     const int cn = c + NS;
@@ -989,6 +996,12 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         // ------------------------------------- B: every score arrived --
         mbar_wait_bounded<true>(bar_score, 0, p.err, 4, kWaitNs);
         stampk(p.stamp_slot, 4);                 // every CTA's scores here
+        if (kAttend && tid == 32) {
+            // the copies' descriptors again, a top-K ahead of the first copy
+            // (fetched at entry, which can be microseconds earlier)
+            prefetch_tensormap(&tmk);
+            prefetch_tensormap(&tmv);
+        }
 
         // --------------------------------------------------- C: select --
         float2 rv[16];                       // C <= 16: a tree, not a chain
@@ -1159,6 +1172,7 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         // the first copies)
         fence_proxy_async_smem();
         __syncwarp();
+        stampk(p.stamp_slot, 23);                // proxy fence passed
         int vbuf0 = cnt_w > 0 ? issue(0) : 0;
         int vbuf1 = npbuf == 2 && cnt_w > 1 ? issue(1) : 0;
         stampk(p.stamp_slot, 15);                // first page copies issued

@@ -24,11 +24,14 @@ import numpy as np
 
 from . import build
 
-NAMES = {0: "entry", 1: "released", 2: "query+weights", 3: "own rows scored",
+NAMES = {0: "entry (before the release: negative)", 1: "released", 2: "query+weights", 3: "own rows scored",
          4: "all scores", 5: "top-K", 6: "1st page landed", 7: "attended",
          8: "warp merge", 9: "cluster merge", 10: "output written"}
-SUB = {11: "histogram", 12: "boundary bin", 13: "ballot", 14: "ranked", 5: "top-K done",
-       16: "barrier", 17: "page ids", 15: "copies issued"}
+SUB = {21: "warp 0 histogram issued", 11: "histogram", 12: "boundary bin",
+       22: "warp 0 ballot words out", 13: "ballot", 14: "ranked", 5: "top-K done",
+       16: "barrier", 17: "page ids", 23: "proxy fence", 15: "copies issued"}
+SCORE = {18: "scoring starts", 19: "first code stage here", 20: "warp 0 scored first stage",
+         3: "own rows scored"}
 
 
 def main(argv) -> None:
@@ -112,7 +115,7 @@ def main(argv) -> None:
     print()
     print("| stamp (globaltimer from release) | median CTA (ns) | slowest CTA (ns) |")
     print("|---|---|---|")
-    for j in range(1, 11):
+    for j in range(0, 11):
         med, mx = [], []
         for k in slots:
             t = T[k, :ncta]
@@ -132,6 +135,42 @@ def main(argv) -> None:
             if not ok.any():
                 continue
             dd = (c[ok, j] - c[ok, 4]) / ghz
+            med.append(np.median(dd))
+            mx.append(dd.max())
+        if med:
+            print(f"| {name} | {np.median(med):.0f} | {np.median(mx):.0f} |")
+    print()
+    # the same phases by the KV head's block size (CTA i of a launch works
+    # on head (i / C) % Hkv, C CTAs per head)
+    pairs = layers[0].data.num_seqs * layers[0].data.num_kv_heads
+    per_head = max(1, ncta // pairs)
+    hkv = layers[0].data.num_kv_heads
+    print("| phase | " + " | ".join(f"bs {b}: median CTA (ns)" for b in (16, 32, 64)) + " |")
+    print("|---|---|---|---|")
+    for j in range(2, 11):
+        cols = []
+        for b in (16, 32, 64):
+            med = []
+            for k in slots:
+                bsz = np.asarray(layers[k].data.block_size)
+                ctas = [i for i in range(ncta) if int(bsz[(i // per_head) % hkv]) == b]
+                if not ctas:
+                    continue
+                c = Cc[k, ctas]
+                med.append(np.median((c[:, j] - c[:, j - 1]) / ghz))
+            cols.append(f"{np.median(med):.0f}" if med else "-")
+        print(f"| {NAMES[j - 1]} -> {NAMES[j]} | " + " | ".join(cols) + " |")
+    print()
+    print("| scoring sub-phase (clock64 from 'query+weights') | median CTA (ns) | slowest CTA (ns) |")
+    print("|---|---|---|")
+    for j, name in SCORE.items():
+        med, mx = [], []
+        for k in slots:
+            c = Cc[k, :ncta]
+            ok = c[:, j] != 0
+            if not ok.any():
+                continue
+            dd = (c[ok, j] - c[ok, 2]) / ghz
             med.append(np.median(dd))
             mx.append(dd.max())
         if med:
