@@ -1419,31 +1419,10 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         mbar_wait_bounded<true>(bar_merge, 0, p.err, 3, kWaitNs);
         stampk(p.stamp_slot, 9);                 // every CTA's partial slice here
         __syncthreads();                                    // this CTA's own stores
-        // per (row, partial) weight exp2(M_r - M) / L: one thread per pair
-        // (G * C <= 256), the C partials of a row on C consecutive lanes
-        // reduced by shuffles; then two channels of one row per thread
-        float* fac = reinterpret_cast<float*>(regB);   // [G][C]; the warp partials are consumed
-        {
-            const int pairs = G << lgC;
-            if (tid < ((pairs + 31) & ~31)) {             // whole warps (full-mask shuffles)
-                const bool act = tid < pairs;
-                const int row = act ? tid >> lgC : 0, r = act ? tid & (static_cast<int>(C) - 1) : 0;
-                const float2 ml = act ? *reinterpret_cast<const float2*>(&recvML[(r * G + row) * 2])
-                                      : make_float2(-INFINITY, 0.0f);
-                float M = ml.x;
-                for (int o = 1; o < static_cast<int>(C); o <<= 1)
-                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-                const float e = M != -INFINITY ? fast_exp2(ml.x - M) : 0.0f;
-                float L = ml.y * e;
-                for (int o = 1; o < static_cast<int>(C); o <<= 1)
-                    L += __shfl_xor_sync(0xffffffffu, L, o);
-                if (act) fac[(row << lgC) + r] = L > 0.0f ? e * fast_rcp(L) : 0.0f;
-            }
-        }
-        __syncthreads();
-        // two channels of one row per 4 consecutive lanes, each lane summing
-        // every 4th partial, then a 2-step shuffle: each output takes C/4
-        // dependent steps instead of C
+        // two channels of one row per 4 consecutive lanes, each lane taking
+        // every 4th partial: the row's M and L and the weighted sums are
+        // reduced over the 4 lanes by 2-step shuffles (no block barrier
+        // between the weights and the sums)
         const int tot = G * ds * 2;
         for (int base = 0; base < tot; base += kThreads) {
             if (base + (tid & ~31) >= tot) break;     // whole warps (full-mask shuffles)
@@ -1451,22 +1430,40 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
             const bool act = idx < tot;
             const int pr = act ? idx >> 2 : 0, qtr = idx & 3;
             const int row = pr >> (lgds - 1), dl = (pr & (ds / 2 - 1)) * 2;
-            const float* fr = fac + (row << lgC);
-            float a0 = 0.0f, a1 = 0.0f;
+            float2 ml[4];
+            float M = -INFINITY;
 #pragma unroll
-            for (int r4 = 0; r4 < 16; r4 += 4) {
-                const int r = r4 + qtr;
+            for (int j = 0; j < 4; ++j) {
+                const int r = 4 * j + qtr;
+                ml[j] = act && r < static_cast<int>(C)
+                            ? *reinterpret_cast<const float2*>(&recvML[(r * G + row) * 2])
+                            : make_float2(-INFINITY, 0.0f);
+                M = fmaxf(M, ml[j].x);
+            }
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+            float L = 0.0f, a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = 4 * j + qtr;
                 if (act && r < static_cast<int>(C)) {
+                    const float e = M != -INFINITY ? fast_exp2(ml[j].x - M) : 0.0f;
+                    L = fmaf(ml[j].y, e, L);
                     const float2 v =
                         *reinterpret_cast<const float2*>(&recvO[(r * G + row) * ds + dl]);
-                    a0 = fmaf(v.x, fr[r], a0);
-                    a1 = fmaf(v.y, fr[r], a1);
+                    a0 = fmaf(v.x, e, a0);
+                    a1 = fmaf(v.y, e, a1);
                 }
             }
+            L += __shfl_xor_sync(0xffffffffu, L, 1);
             a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
             a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+            L += __shfl_xor_sync(0xffffffffu, L, 2);
             a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
             a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+            const float rl = L > 0.0f ? fast_rcp(L) : 0.0f;
+            a0 *= rl;
+            a1 *= rl;
             if (act && qtr == 0)
                 *reinterpret_cast<uint32_t*>(outp + row * kD + rank * ds + dl) = pack_bf16x2(a0, a1);
         }
