@@ -1315,30 +1315,38 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         // of every row, receives that slice of every CTA's partial (16-byte
         // asynchronous stores counted on its mbarrier, its own by plain
         // stores), merges the C partials and writes the slice.
-        __syncthreads();                                   // page buffers are dead
-        float* Ow = reinterpret_cast<float*>(regB);        // [warps][G][128]
-        float* mw = Ow + kWarps * G * kD;                  // [warps][G]
-        float* lw = mw + kWarps * G;
+        // Warp partials: with G <= 8 each warp writes its partial (O rows,
+        // then (M, L) pairs) into its own page buffers, which only it used,
+        // so no block barrier is needed first; a wider group's partials
+        // span the page buffers of several warps and wait for all of them.
+        constexpr int kWarpStride = NPB * kPageSmem / 4;   // floats
+        float* Ow = reinterpret_cast<float*>(regB);
+        auto ow_at = [&](int w, int row) -> float* {
+            return BIG_GROUP ? Ow + (w * G + row) * kD : Ow + w * kWarpStride + row * kD;
+        };
+        auto ml_at = [&](int w, int row) -> float* {
+            return BIG_GROUP ? Ow + kWarps * G * kD + (w * G + row) * 2
+                             : Ow + w * kWarpStride + G * kD + row * 2;
+        };
+        if constexpr (BIG_GROUP) {
+            __syncthreads();                               // page buffers are dead
+        } else {
+            __syncwarp();                                  // this warp's reads of them are done
+        }
         if (g < G) {
+            float* orow = ow_at(warp, g);
 #pragma unroll
             for (int t = 0; t < 16; ++t)
-                *reinterpret_cast<float2*>(&Ow[(warp * G + g) * kD + t * 8 + 2 * t4]) =
-                    make_float2(o[t][0], o[t][1]);
-            if (t4 == 0) {
-                mw[warp * G + g] = m0;
-                lw[warp * G + g] = l0;
-            }
+                *reinterpret_cast<float2*>(&orow[t * 8 + 2 * t4]) = make_float2(o[t][0], o[t][1]);
+            if (t4 == 0) *reinterpret_cast<float2*>(ml_at(warp, g)) = make_float2(m0, l0);
         }
         if constexpr (BIG_GROUP) {
             if (g + 8 < G) {
+                float* orow = ow_at(warp, g + 8);
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
-                    *reinterpret_cast<float2*>(&Ow[(warp * G + g + 8) * kD + t * 8 + 2 * t4]) =
-                        make_float2(o[t][2], o[t][3]);
-                if (t4 == 0) {
-                    mw[warp * G + g + 8] = m8;
-                    lw[warp * G + g + 8] = l8;
-                }
+                    *reinterpret_cast<float2*>(&orow[t * 8 + 2 * t4]) = make_float2(o[t][2], o[t][3]);
+                if (t4 == 0) *reinterpret_cast<float2*>(ml_at(warp, g + 8)) = make_float2(m8, l8);
             }
         }
         __syncthreads();
@@ -1350,20 +1358,20 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         // place by every thread of the row (a row with no valid token has
         // M = -inf and gets zero weights)
         auto cta_partial = [&](int row, int d, float& M, float& L) -> float4 {
-            float mv[kWarps];
+            float2 mv[kWarps];
             M = -INFINITY;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
-                mv[w] = mw[w * G + row];
-                M = fmaxf(M, mv[w]);
+                mv[w] = *reinterpret_cast<const float2*>(ml_at(w, row));
+                M = fmaxf(M, mv[w].x);
             }
             L = 0.0f;
             float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
-                const float e = M != -INFINITY ? fast_exp2(mv[w] - M) : 0.0f;
-                L = fmaf(lw[w * G + row], e, L);
-                const float4 v = *reinterpret_cast<const float4*>(&Ow[(w * G + row) * kD + d]);
+                const float e = M != -INFINITY ? fast_exp2(mv[w].x - M) : 0.0f;
+                L = fmaf(mv[w].y, e, L);
+                const float4 v = *reinterpret_cast<const float4*>(ow_at(w, row) + d);
                 a.x = fmaf(v.x, e, a.x);
                 a.y = fmaf(v.y, e, a.y);
                 a.z = fmaf(v.z, e, a.z);
