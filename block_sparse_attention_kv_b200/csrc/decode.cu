@@ -674,10 +674,9 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
     auto stage_buf = [&](int st) -> uint8_t* { return regB + p.ring_off + st * kStageBytes; };
     if (tid == 0) {
         if (kAttend && C > 1)
-            // every other CTA's slice of its partial: G rows x 128/C
-            // channels, and (M, L) per row
-            mbar_arrive_expect_tx(smem_u32(&sm.bar_merge),
-                                  (C - 1) * (G * (kD / C) * 4 + 8 * G));
+            // every CTA's slice of its partial, this one's own included:
+            // G rows x 128/C channels, and (M, L) per row
+            mbar_arrive_expect_tx(smem_u32(&sm.bar_merge), C * (G * (kD / C) * 4 + 8 * G));
         if (kSelect && (MODE != kModeSelect || rank == 0))
             // every CTA's scores but this one's own (plain stores), and
             // every CTA's (min, max)
@@ -1405,28 +1404,21 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
             const float4 a = cta_partial(row, d, M, L);
             const uint32_t owner = static_cast<uint32_t>(d >> lgds);
             float* dst = &recvO[(rank * G + row) * ds + (d - static_cast<int>(owner) * ds)];
-            if (owner == rank)
-                *reinterpret_cast<float4*>(dst) = a;
-            else
-                st_async_v4(dsmem_addr(smem_u32(dst), owner), a.x, a.y, a.z, a.w,
-                            dsmem_addr(bar_merge, owner));
+            // to every owner by st.async, this CTA included, so that the
+            // owner's mbarrier covers its own slice too (no block barrier)
+            st_async_v4(dsmem_addr(smem_u32(dst), owner), a.x, a.y, a.z, a.w,
+                        dsmem_addr(bar_merge, owner));
             if (d4 < static_cast<int>(C)) {   // the row's (M, L) to owner d4
                 const uint32_t o = static_cast<uint32_t>(d4);
                 float* ml = &recvML[(rank * G + row) * 2];
-                if (o == rank) {
-                    ml[0] = M;
-                    ml[1] = L;
-                } else {
-                    st_async_v2(dsmem_addr(smem_u32(ml), o), M, L, dsmem_addr(bar_merge, o));
-                }
+                st_async_v2(dsmem_addr(smem_u32(ml), o), M, L, dsmem_addr(bar_merge, o));
             }
         }
-        // every other CTA's slice of its partial has arrived (each sends only
+        // every CTA's slice of its partial has arrived (each sends only
         // after its own page lookups, so no CTA leaves while another may
         // still read its staged page ids)
         mbar_wait_bounded<true>(bar_merge, 0, p.err, 3, kWaitNs);
         stampk(p.stamp_slot, 9);                 // every CTA's partial slice here
-        __syncthreads();                                    // this CTA's own stores
         // two channels of one row per 4 consecutive lanes, each lane taking
         // every 4th partial: the row's M and L and the weighted sums are
         // reduced over the 4 lanes by 2-step shuffles (no block barrier
