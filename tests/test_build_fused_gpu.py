@@ -85,3 +85,52 @@ def test_fused_matches_the_oracle_on_the_llama_layer(lib):
                          zp.cpu().numpy())
         rep.heads += 1
     assert rep.code_mismatch == 0 and rep.param_mismatch == 0, rep.notes[:5]
+
+
+def test_one_call_codes_on_exact_half_steps(lib):
+    """Steps 1-2 on exact ties of c / scale, built from the keys: every
+    block holds one key value per channel, placed at j / 2 steps of a
+    per-channel step e (min at j = 0, max at j = 30, so scale = e and
+    c / scale = offset + j / 2), so odd j give exact half-integers (about
+    half of the 40,960 codes), which round half to even.  The one call
+    must equal the two calls and the oracle bit for bit."""
+    abi, pipeline = lib
+    w = synth.custom("half_steps", 1, 8, 2, [4096], [16, 64], 1024, seed=44)
+    d = synth.make_layer(w, 0, "cuda")
+    rng = np.random.default_rng(9)
+    P, D = synth.PAGE_SIZE, 128
+    L = int(d.seq_lens[0])
+    npg = L // P
+    kk = np.empty((npg * P, d.num_kv_heads, D), dtype=np.float32)
+    for h in range(d.num_kv_heads):
+        bs = int(d.block_size[h])
+        nb = L // bs
+        for ch in range(D):
+            e = 2.0 ** -(4 + ch % 3)
+            off = (ch % 5 - 2) * 3 * e
+            j = rng.integers(0, 31, nb)
+            j[0], j[1] = 0, 30
+            vals = off + j * e / 2
+            kk[:, h, ch] = np.repeat(vals, bs)[: npg * P]
+    kb = torch.from_numpy(kk).to("cuda").to(torch.bfloat16)
+    assert torch.equal(kb.float().cpu(), torch.from_numpy(kk))   # every key exact in bf16
+    ids = d.page_table[0, :npg].long()
+    d.k_pages[ids] = kb.view(npg, P, d.num_kv_heads, D).permute(0, 2, 1, 3)
+    a = pipeline.DeviceLayer(d)
+    b = pipeline.DeviceLayer(d)
+    a.build_centroids()
+    b.cent.codes.fill_(0xAB)
+    b.build_centroids(fused=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a.cent.codes, b.cent.codes)
+    assert torch.equal(a.cent.scale.view(torch.int32), b.cent.scale.view(torch.int32))
+    assert torch.equal(a.cent.zp, b.cent.zp)
+    host = synth.host_layer(d)
+    for h in range(d.num_kv_heads):
+        bs = int(d.block_size[h])
+        keys = O.gather_head_tokens(host.k_bits, host.page_table[0], L, h)
+        want = O.quantize_centroids(O.build_centroids(keys, bs))
+        n = want.codes.shape[0]
+        got = O.unpack_codes(b.codes_of(0, h, n).cpu().numpy())
+        assert np.array_equal(got, want.codes), h
+        assert np.array_equal(want.scale, np.exp2(-(4 + np.arange(D) % 3)).astype(np.float32))
