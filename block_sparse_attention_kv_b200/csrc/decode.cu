@@ -1312,8 +1312,8 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         // Warps merge in shared memory into this CTA's partial (O, M, L);
         // with C > 1 CTA r owns output channels [r * 128/C, (r + 1) * 128/C)
         // of every row, receives that slice of every CTA's partial (16-byte
-        // asynchronous stores counted on its mbarrier, its own by plain
-        // stores), merges the C partials and writes the slice.
+        // asynchronous stores counted on its mbarrier, its own included),
+        // merges the C partials and writes the slice.
         // Warp partials: with G <= 8 each warp writes its partial (O rows,
         // then (M, L) pairs) into its own page buffers, which only it used,
         // so no block barrier is needed first; a wider group's partials
