@@ -859,8 +859,12 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
                     }
                 }
                 if (c == 0) stampk(p.stamp_slot, 20);  // warp 0 scored the first stage
+                // a stage buffer is refilled once every warp is done with it
+                // (uniform); the block barrier after the loop, before the
+                // scores are read, covers the stages that are not refilled
+                if (c + NS >= nchunks) continue;
                 __syncthreads();
-                if (tid == 0 && c + NS < nchunks) {
+                if (tid == 0) {
                     const int cn = c + NS;
                     const int rows_n = min(kSRows, nrows - cn * kSRows);
                     const uint32_t bar = smem_u32(&sm.bar_code[stage]);
