@@ -366,11 +366,16 @@ __device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int
         extract_bitmap_long(bitmap, j0, j1, pos, out, lo, hi);
         return;
     }
+    // the run's words read first (independent loads), then placed in order
     const uint32_t lt = (1u << lane) - 1u;
-    for (int j = j0; j < j1 && static_cast<int>(pos) < hi; ++j) {
-        const uint32_t bits = bitmap[j];
+    uint32_t wb[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) wb[u] = j0 + u < j1 ? bitmap[j0 + u] : 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t bits = wb[u];
         const int at = static_cast<int>(pos + __popc(bits & lt));
-        if (((bits >> lane) & 1u) && at >= lo && at < hi) out[at - lo] = j * 32 + lane;
+        if (((bits >> lane) & 1u) && at >= lo && at < hi) out[at - lo] = (j0 + u) * 32 + lane;
         pos += __popc(bits);
     }
 }
