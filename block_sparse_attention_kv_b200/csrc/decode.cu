@@ -528,10 +528,15 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                         const uint32_t key = lane < m ? ckey[lane] : 0u;
                         const int idx = lane < m ? cidx[lane] : 0x7fffffff;
                         int rank = 0;
-                        for (int j = 0; j < m; ++j) {
-                            const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
-                            const int ij = __shfl_sync(0xffffffffu, idx, j);
-                            rank += (kj > key) || (kj == key && ij < idx);
+                        // 8 candidates per step, their shuffles independent
+                        for (int jb = 0; jb < m; jb += 8) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int j = jb + u;   // < 32 (m <= 32)
+                                const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+                                const int ij = __shfl_sync(0xffffffffu, idx, j);
+                                rank += j < m && ((kj > key) || (kj == key && ij < idx));
+                            }
                         }
                         if (lane < m && rank < need) {
                             atomicOr(&inw[idx >> 5], 1u << (idx & 31));
@@ -754,12 +759,19 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         if (tid < kD) {
             const __nv_bfloat16* qh = p.q + (static_cast<int64_t>(s) * p.kv.Hq + h * G) * kD + tid;
             // the group's queries are read once (they may live in host
-            // memory) and kept for the attention phase
+            // memory), all loads issued before the first use, and kept for
+            // the attention phase; qbar sums them in head order
+            constexpr int kQMax = BIG_GROUP ? 16 : 8;
+            __nv_bfloat16 qv[kQMax];
+#pragma unroll
+            for (int j = 0; j < kQMax; ++j) qv[j] = j < G ? qh[j * kD] : __float2bfloat16(0.0f);
             float qb = 0.0f;
-            for (int j = 0; j < G; ++j) {
-                const __nv_bfloat16 qv = qh[j * kD];
-                qs[j * kD + tid] = qv;
-                qb += __bfloat162float(qv);
+#pragma unroll
+            for (int j = 0; j < kQMax; ++j) {
+                if (j < G) {
+                    qs[j * kD + tid] = qv[j];
+                    qb += __bfloat162float(qv[j]);
+                }
             }
             const float wv = BF16C ? qb : qb * scl;
             sm.w[tid] = wv;
