@@ -380,6 +380,15 @@ __device__ __forceinline__ void block_extract_bitmap(const uint32_t* bitmap, int
     }
 }
 
+// The warp that owns ballot word wd when warps own runs of wpw words:
+// counted against the run starts instead of a division on the select's path.
+__device__ __forceinline__ int word_owner(int wd, int wpw) {
+    int w = 0;
+#pragma unroll
+    for (int u = 1; u < kWarps; ++u) w += wd >= u * wpw;
+    return w;
+}
+
 // Top-k of sc[0..n) (largest scores, ties to the lower index) in ascending
 // index order; only list entries [lo, hi) are written, to out[0 .. hi-lo).
 // [mn, mx] is the range of the scores.  The kBins histogram bins at the
@@ -540,7 +549,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                         }
                         if (lane < m && rank < need) {
                             atomicOr(&inw[idx >> 5], 1u << (idx & 31));
-                            atomicAdd(&sm.scan[(idx >> 5) / wpw], 1u);
+                            atomicAdd(&sm.scan[word_owner(idx >> 5, wpw)], 1u);
                         }
                     }
                 } else {
@@ -554,7 +563,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
                         }
                         if (rank < need) {
                             atomicOr(&inw[idx >> 5], 1u << (idx & 31));
-                            atomicAdd(&sm.scan[(idx >> 5) / wpw], 1u);
+                            atomicAdd(&sm.scan[word_owner(idx >> 5, wpw)], 1u);
                         }
                     }
                 }
@@ -840,10 +849,12 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
         // 8-lane group's scores of rows r4 .. r4 + 3 of a stage (values for
         // rows past `rows` are discarded here).
         auto chunk_loop = [&](auto&& score4) {
+            // ring stage and mbarrier phase of chunk c, counted (NS is a
+            // launch value: a division here sat on the critical path)
+            int stage = 0, phase = 0;
 #pragma unroll 1
             for (int c = 0; c < nchunks; ++c) {
-                const int stage = c % NS;
-                mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), (c / NS) & 1, p.err, 1, kWaitNs);
+                mbar_wait_bounded(smem_u32(&sm.bar_code[stage]), phase, p.err, 1, kWaitNs);
                 if (c == 0) stampk(p.stamp_slot, 19);  // first code stage here
                 const int rows = min(kSRows, nrows - c * kSRows);
                 const uint8_t* sbuf = stage_buf(stage);
@@ -879,15 +890,20 @@ __global__ void __launch_bounds__(kThreads, NPB == 2 ? 1 : ABSP_DECODE_MIN_BLOCK
                 // a stage buffer is refilled once every warp is done with it
                 // (uniform); the block barrier after the loop, before the
                 // scores are read, covers the stages that are not refilled
-                if (c + NS >= nchunks) continue;
-                __syncthreads();
-                if (tid == 0) {
-                    const int cn = c + NS;
-                    const int rows_n = min(kSRows, nrows - cn * kSRows);
-                    const uint32_t bar = smem_u32(&sm.bar_code[stage]);
-                    fence_proxy_async_smem();
-                    mbar_arrive_expect_tx(bar, rows_n * kRow);
-                    bulk_g2s(smem_u32(sbuf), cbase + cn * kStageBytes, rows_n * kRow, bar);
+                if (c + NS < nchunks) {
+                    __syncthreads();
+                    if (tid == 0) {
+                        const int cn = c + NS;
+                        const int rows_n = min(kSRows, nrows - cn * kSRows);
+                        const uint32_t bar = smem_u32(&sm.bar_code[stage]);
+                        fence_proxy_async_smem();
+                        mbar_arrive_expect_tx(bar, rows_n * kRow);
+                        bulk_g2s(smem_u32(sbuf), cbase + cn * kStageBytes, rows_n * kRow, bar);
+                    }
+                }
+                if (++stage == NS) {
+                    stage = 0;
+                    phase ^= 1;
                 }
             }
         };
