@@ -414,7 +414,137 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
         compact_by_threshold(sc, n, order_key(mx), k, out, lo, hi, sm);
         return;
     }
-    if (inv < INFINITY) {
+    // the boundary bin from the histogram (block scan, two barriers):
+    // sm.misc = {bin, scores still needed from it, its count}; the
+    // candidate counter sm.misc[3] reset
+    auto find_boundary = [&]() {
+        {
+            // thread t owns bins 4(255-t) .. 4(255-t)+3 (one 16-byte load);
+            // an exclusive scan in thread order counts the scores above them
+            const uint4 hv = reinterpret_cast<const uint4*>(hist)[255 - tid];
+            const uint32_t tot = hv.x + hv.y + hv.z + hv.w;
+            const uint32_t above = block_excl_scan(tot, sm.scan);
+            if (above < static_cast<uint32_t>(k) && static_cast<uint32_t>(k) <= above + tot) {
+                const uint32_t c[4] = {hv.w, hv.z, hv.y, hv.x};  // descending bins
+                uint32_t cum = above;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (cum < static_cast<uint32_t>(k) && static_cast<uint32_t>(k) <= cum + c[j]) {
+                        sm.misc[0] = 4 * (255 - tid) + 3 - j;
+                        sm.misc[1] = k - static_cast<int>(cum);
+                        sm.misc[2] = static_cast<int>(c[j]);
+                    }
+                    cum += c[j];
+                }
+            }
+            if (tid == 32) sm.misc[3] = 0;
+        }
+        __syncthreads();
+    };
+    // exact rank among the m candidates: larger key first, ties to the
+    // lower index; the `need` best join the selection (bitmap words and the
+    // owning warps' counts); ends with a block barrier
+    auto rank_candidates = [&](int m, int need, int wpw) {
+        if (m <= 32) {
+            if (warp == 0) {
+                const uint32_t key = lane < m ? ckey[lane] : 0u;
+                const int idx = lane < m ? cidx[lane] : 0x7fffffff;
+                int rank = 0;
+                // 8 candidates per step, their shuffles independent
+                for (int jb = 0; jb < m; jb += 8) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = jb + u;   // < 32 (m <= 32)
+                        const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+                        const int ij = __shfl_sync(0xffffffffu, idx, j);
+                        rank += j < m && ((kj > key) || (kj == key && ij < idx));
+                    }
+                }
+                if (lane < m && rank < need) {
+                    atomicOr(&inw[idx >> 5], 1u << (idx & 31));
+                    atomicAdd(&sm.scan[word_owner(idx >> 5, wpw)], 1u);
+                }
+            }
+        } else {
+            for (int c = tid; c < m; c += kThreads) {
+                const uint32_t key = ckey[c];
+                const int idx = cidx[c];
+                int rank = 0;
+                for (int j = 0; j < m; ++j) {
+                    const uint32_t kj = ckey[j];
+                    rank += (kj > key) || (kj == key && cidx[j] < idx);
+                }
+                if (rank < need) {
+                    atomicOr(&inw[idx >> 5], 1u << (idx & 31));
+                    atomicAdd(&sm.scan[word_owner(idx >> 5, wpw)], 1u);
+                }
+            }
+        }
+        __syncthreads();
+    };
+    if (inv < INFINITY && n <= 8 * kThreads) {
+        // Up to 2048 scores: thread t holds scores 8t .. 8t+7 in registers
+        // (histogram and selection in one load) and writes byte t of the
+        // selection bitmap, so warp w owns words 8w .. 8w+7 and no warp vote
+        // is needed; candidates take their slots by one atomic per thread
+        // that has any (their order does not matter to the ranking).
+        const int i0 = 8 * tid;
+        float x[8];
+        int bn[8];
+        if (i0 + 8 <= n) {
+            const float4 a = reinterpret_cast<const float4*>(sc)[2 * tid];
+            const float4 b = reinterpret_cast<const float4*>(sc)[2 * tid + 1];
+            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+            x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+        } else {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) x[v] = i0 + v < n ? sc[i0 + v] : mn;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) bn[v] = i0 + v < n ? value_bin(x[v], mn, inv) : -1;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+            if (bn[v] >= 0) atomicAdd(&hist[bn[v]], 1u);
+        stampk(stamp_slot, 21);                  // this thread's histogram updates issued
+        __syncthreads();
+        stampk(stamp_slot, 11);                  // histogram done
+        find_boundary();
+        const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
+        stampk(stamp_slot, 12);                  // boundary bin known
+        if (m <= kMaxCand) {
+            const bool all_in = need == m;
+            uint32_t selb = 0u, candb = 0u;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int b = bn[v];
+                if (b > bstar || (all_in && b == bstar)) selb |= 1u << v;
+                else if (b == bstar) candb |= 1u << v;
+            }
+            reinterpret_cast<uint8_t*>(inw)[tid] = static_cast<uint8_t>(selb);
+            const uint32_t cnt = __reduce_add_sync(0xffffffffu, __popc(selb));
+            if (lane == 0) sm.scan[warp] = cnt;
+            if (candb != 0u) {
+                int pos = atomicAdd(&sm.misc[3], __popc(candb));
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    if ((candb >> v) & 1u) {
+                        ckey[pos] = order_key(x[v]);
+                        cidx[pos] = i0 + v;
+                        ++pos;
+                    }
+                }
+            }
+            stampk(stamp_slot, 22);              // this thread's bitmap byte out
+            __syncthreads();
+            stampk(stamp_slot, 13);              // bitmap and candidates out
+            if (!all_in) rank_candidates(m, need, 8);
+            stampk(stamp_slot, 14);              // boundary candidates ranked
+            block_extract_bitmap(inw, (n + 31) / 32, 8, sm.scan, out, lo, hi);
+            __syncthreads();
+            return;
+        }
+        __syncthreads();
+    } else if (inv < INFINITY) {
         // histogram of the scores over kBins equal bins of [mn, mx] (the
         // bins were zeroed by the caller).  Warp w owns the ballot words
         // [w * wpw, (w + 1) * wpw) (32 scores each) here and in the ballot
@@ -450,28 +580,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
         stampk(stamp_slot, 21);                  // warp 0's histogram updates issued
         __syncthreads();
         stampk(stamp_slot, 11);                  // histogram done
-        {
-            // thread t owns bins 4(255-t) .. 4(255-t)+3 (one 16-byte load);
-            // an exclusive scan in thread order counts the scores above them
-            const uint4 hv = reinterpret_cast<const uint4*>(hist)[255 - tid];
-            const uint32_t tot = hv.x + hv.y + hv.z + hv.w;
-            const uint32_t above = block_excl_scan(tot, sm.scan);
-            if (above < static_cast<uint32_t>(k) && static_cast<uint32_t>(k) <= above + tot) {
-                const uint32_t c[4] = {hv.w, hv.z, hv.y, hv.x};  // descending bins
-                uint32_t cum = above;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (cum < static_cast<uint32_t>(k) && static_cast<uint32_t>(k) <= cum + c[j]) {
-                        sm.misc[0] = 4 * (255 - tid) + 3 - j;
-                        sm.misc[1] = k - static_cast<int>(cum);
-                        sm.misc[2] = static_cast<int>(c[j]);
-                    }
-                    cum += c[j];
-                }
-            }
-            if (tid == 32) sm.misc[3] = 0;
-        }
-        __syncthreads();
+        find_boundary();
         const int bstar = sm.misc[0], need = sm.misc[1], m = sm.misc[2];
         stampk(stamp_slot, 12);                  // boundary bin known
         if (m <= kMaxCand) {
@@ -529,46 +638,7 @@ __device__ __forceinline__ void block_topk(const float* sc, int n, int k, float 
             stampk(stamp_slot, 22);              // warp 0's ballot words out
             __syncthreads();
             stampk(stamp_slot, 13);              // ballot words and candidates out
-            if (!all_in) {
-                // exact rank among the candidates: larger key first, ties to
-                // the lower index; the `need` best join the selection
-                if (m <= 32) {
-                    if (warp == 0) {
-                        const uint32_t key = lane < m ? ckey[lane] : 0u;
-                        const int idx = lane < m ? cidx[lane] : 0x7fffffff;
-                        int rank = 0;
-                        // 8 candidates per step, their shuffles independent
-                        for (int jb = 0; jb < m; jb += 8) {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int j = jb + u;   // < 32 (m <= 32)
-                                const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
-                                const int ij = __shfl_sync(0xffffffffu, idx, j);
-                                rank += j < m && ((kj > key) || (kj == key && ij < idx));
-                            }
-                        }
-                        if (lane < m && rank < need) {
-                            atomicOr(&inw[idx >> 5], 1u << (idx & 31));
-                            atomicAdd(&sm.scan[word_owner(idx >> 5, wpw)], 1u);
-                        }
-                    }
-                } else {
-                    for (int c = tid; c < m; c += kThreads) {
-                        const uint32_t key = ckey[c];
-                        const int idx = cidx[c];
-                        int rank = 0;
-                        for (int j = 0; j < m; ++j) {
-                            const uint32_t kj = ckey[j];
-                            rank += (kj > key) || (kj == key && cidx[j] < idx);
-                        }
-                        if (rank < need) {
-                            atomicOr(&inw[idx >> 5], 1u << (idx & 31));
-                            atomicAdd(&sm.scan[word_owner(idx >> 5, wpw)], 1u);
-                        }
-                    }
-                }
-                __syncthreads();
-            }
+            if (!all_in) rank_candidates(m, need, wpw);
             stampk(stamp_slot, 14);              // boundary candidates ranked
             block_extract_bitmap(inw, nwords, wpw, sm.scan, out, lo, hi);
             __syncthreads();
