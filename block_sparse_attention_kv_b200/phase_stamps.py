@@ -28,7 +28,7 @@ NAMES = {0: "entry (before the release: negative)", 1: "released", 2: "query+wei
          4: "all scores", 5: "top-K", 6: "1st page landed", 7: "attended",
          8: "warp merge", 9: "cluster merge", 10: "output written"}
 SUB = {21: "warp 0 histogram issued", 11: "histogram", 12: "boundary bin",
-       22: "warp 0 ballot words out", 13: "ballot", 14: "ranked", 5: "top-K done",
+       22: "warp 0 selection words out", 13: "selection words and candidates", 14: "ranked", 5: "top-K done",
        16: "barrier", 17: "page ids", 23: "proxy fence", 15: "copies issued"}
 SCORE = {18: "scoring starts", 19: "first code stage here", 20: "warp 0 scored first stage",
          3: "own rows scored"}
@@ -102,80 +102,79 @@ def main(argv) -> None:
     slots = range(4, min(L, 64))
     print(json.dumps({"workload": wname, "layers": L, "us_per_launch_stamped": round(us, 3),
                       "ctas": ncta, "sm_ghz": ghz, "build_id": abi.absp_build_id()}))
-    print("| phase | median CTA (ns) | slowest CTA (ns) |")
-    print("|---|---|---|")
+    pairs = layers[0].data.num_seqs * layers[0].data.num_kv_heads
+    block_sizes = [np.asarray(layers[k].data.block_size) for k in range(L)]
+    for line in tables(T, Cc, ncta, ghz, slots, block_sizes, max(1, ncta // pairs)):
+        print(line)
+
+
+def _row(name: str, med: list, mx: list) -> str:
+    return f"| {name} | {np.median(med):.0f} | {np.median(mx):.0f} |"
+
+
+def tables(T, Cc, ncta: int, ghz: float, slots, block_sizes, per_head: int) -> list[str]:
+    """The timeline tables as markdown lines.
+
+    T[k, i, j] is the globaltimer stamp (ns) and Cc[k, i, j] the clock64
+    stamp of slot j by CTA i in launch k (0 where the slot was not
+    stamped); `slots` are the launches summarised; block_sizes[k] is launch
+    k's per-KV-head block-size table, and CTA i works on KV head
+    (i // per_head) % len(block_sizes[k]).  Each figure is the median over
+    the launches of the median CTA and of the slowest CTA.
+    """
+    out = ["| phase | median CTA (ns) | slowest CTA (ns) |", "|---|---|---|"]
     for j in range(2, 11):
         med, mx = [], []
         for k in slots:
-            c = Cc[k, :ncta]
-            dd = (c[:, j] - c[:, j - 1]) / ghz
+            dd = (Cc[k, :ncta, j] - Cc[k, :ncta, j - 1]) / ghz
             med.append(np.median(dd))
             mx.append(dd.max())
-        print(f"| {NAMES[j - 1]} -> {NAMES[j]} | {np.median(med):.0f} | {np.median(mx):.0f} |")
-    print()
-    print("| stamp (globaltimer from release) | median CTA (ns) | slowest CTA (ns) |")
-    print("|---|---|---|")
+        out.append(_row(f"{NAMES[j - 1]} -> {NAMES[j]}", med, mx))
+    out += ["", "| stamp (globaltimer from release) | median CTA (ns) | slowest CTA (ns) |",
+            "|---|---|---|"]
     for j in range(0, 11):
         med, mx = [], []
         for k in slots:
             t = T[k, :ncta]
-            rel = t[:, 1].min()
-            v = t[:, j] - rel
+            v = t[:, j] - t[:, 1].min()
             med.append(np.median(v))
             mx.append(v.max())
-        print(f"| {NAMES[j]} | {np.median(med):.0f} | {np.median(mx):.0f} |")
-    print()
-    print("| top-K sub-phase (clock64 from 'all scores') | median CTA (ns) | slowest CTA (ns) |")
-    print("|---|---|---|")
-    for j, name in SUB.items():
-        med, mx = [], []
-        for k in slots:
-            c = Cc[k, :ncta]
-            ok = c[:, j] != 0
-            if not ok.any():
-                continue
-            dd = (c[ok, j] - c[ok, 4]) / ghz
-            med.append(np.median(dd))
-            mx.append(dd.max())
-        if med:
-            print(f"| {name} | {np.median(med):.0f} | {np.median(mx):.0f} |")
-    print()
-    # the same phases by the KV head's block size (CTA i of a launch works
-    # on head (i / C) % Hkv, C CTAs per head)
-    pairs = layers[0].data.num_seqs * layers[0].data.num_kv_heads
-    per_head = max(1, ncta // pairs)
-    hkv = layers[0].data.num_kv_heads
-    print("| phase | " + " | ".join(f"bs {b}: median CTA (ns)" for b in (16, 32, 64)) + " |")
-    print("|---|---|---|---|")
+        out.append(_row(NAMES[j], med, mx))
+
+    def sub_table(title: str, names: dict, origin: int) -> list[str]:
+        rows = ["", f"| {title} | median CTA (ns) | slowest CTA (ns) |", "|---|---|---|"]
+        for j, name in names.items():
+            med, mx = [], []
+            for k in slots:
+                c = Cc[k, :ncta]
+                ok = c[:, j] != 0
+                if not ok.any():
+                    continue
+                dd = (c[ok, j] - c[ok, origin]) / ghz
+                med.append(np.median(dd))
+                mx.append(dd.max())
+            if med:
+                rows.append(_row(name, med, mx))
+        return rows
+
+    out += sub_table("top-K sub-phase (clock64 from 'all scores')", SUB, 4)
+    sizes = (16, 32, 64)
+    out += ["", "| phase | " + " | ".join(f"bs {b}: median CTA (ns)" for b in sizes) + " |",
+            "|---|---|---|---|"]
     for j in range(2, 11):
         cols = []
-        for b in (16, 32, 64):
+        for b in sizes:
             med = []
             for k in slots:
-                bsz = np.asarray(layers[k].data.block_size)
-                ctas = [i for i in range(ncta) if int(bsz[(i // per_head) % hkv]) == b]
-                if not ctas:
-                    continue
-                c = Cc[k, ctas]
-                med.append(np.median((c[:, j] - c[:, j - 1]) / ghz))
+                bsz = block_sizes[k]
+                ctas = [i for i in range(ncta) if int(bsz[(i // per_head) % len(bsz)]) == b]
+                if ctas:
+                    c = Cc[k, ctas]
+                    med.append(np.median((c[:, j] - c[:, j - 1]) / ghz))
             cols.append(f"{np.median(med):.0f}" if med else "-")
-        print(f"| {NAMES[j - 1]} -> {NAMES[j]} | " + " | ".join(cols) + " |")
-    print()
-    print("| scoring sub-phase (clock64 from 'query+weights') | median CTA (ns) | slowest CTA (ns) |")
-    print("|---|---|---|")
-    for j, name in SCORE.items():
-        med, mx = [], []
-        for k in slots:
-            c = Cc[k, :ncta]
-            ok = c[:, j] != 0
-            if not ok.any():
-                continue
-            dd = (c[ok, j] - c[ok, 2]) / ghz
-            med.append(np.median(dd))
-            mx.append(dd.max())
-        if med:
-            print(f"| {name} | {np.median(med):.0f} | {np.median(mx):.0f} |")
-
+        out.append(f"| {NAMES[j - 1]} -> {NAMES[j]} | " + " | ".join(cols) + " |")
+    out += sub_table("scoring sub-phase (clock64 from 'query+weights')", SCORE, 2)
+    return out
 
 if __name__ == "__main__":
     main(sys.argv)
