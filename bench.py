@@ -160,11 +160,44 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_text(src: str) -> str:
+    """C/C++/CUDA source without its comments and blank space.
+
+    Comments go (a block comment counts as one space) except inside string
+    and character literals, runs of spaces and tabs become one space (inside
+    literals too), and blank lines go; line breaks between code stay, since
+    a preprocessor directive ends at one.
+    """
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == "/" and src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif c == "/" and src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c and src[j] != "\n":
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    lines = (" ".join(l.split()) for l in "".join(out).split("\n"))
+    return "\n".join(l for l in lines if l)
+
+
 def kernel_source_hash() -> str:
+    """sha256 (16 hex digits) of the decode kernel's code, comments ignored."""
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(code_text(f.read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 

@@ -14,13 +14,15 @@
 //               cluster with asynchronous 16-byte distributed-shared-memory
 //               stores that count down the receiver's mbarrier (its own
 //               scores with plain stores).  Meanwhile the sequence's
-//               page-table row is prefetched into L2.
+//               page-table row is staged in shared memory (or its entries
+//               for the CTA's own rows, when the row does not fit).
 //   B  each CTA waits on its own mbarrier until all n_h scores arrived.
 //   C  select:  every CTA runs the same deterministic top-K (largest scores,
 //               ties to the lower block index): a 1024-bin histogram over the
-//               score range finds the bin holding the K-th score, the few
-//               scores in that bin are ranked exactly, and an ordered
-//               compaction writes the ascending block list.  A 4 x 8-bit
+//               score range finds the bin holding the K-th score, a bitmap
+//               marks the scores above it, the few scores in that bin are
+//               ranked exactly, and each warp writes its bitmap words'
+//               entries of the ascending block list.  A 4 x 8-bit
 //               radix select over order-preserving keys covers degenerate
 //               ranges.  All CTAs hold the same list without another
 //               exchange.
@@ -28,13 +30,17 @@
 //               contiguous 1/C share of those pages.  Each warp owns every
 //               8th page: it loads the (page, head) K and V slices with 2-D
 //               tensor copies (128-byte swizzle, no multicast) on its own
-//               mbarrier, then computes S^T = Q K^T and O += P V on mma.sync
+//               mbarrier into one of its one or two page buffers (two in the
+//               one-CTA-per-SM instance), then computes S^T = Q K^T and O += P V on mma.sync
 //               bf16 tiles with the GQA group as the 16-row M dimension and an
 //               online softmax in fp32; each warp also bulk-prefetches its
 //               next two pages into L2.
-//   E  merge:   warps merge in shared memory; CTAs write their (m, l, O)
-//               partials into CTA 0 through distributed shared memory and
-//               arrive on CTA 0's mbarrier; CTA 0 merges and writes bf16.
+//   E  merge:   warps merge in shared memory into the CTA's partial; CTA r
+//               owns output channels [r*128/C, (r+1)*128/C) and receives
+//               that slice of every CTA's partial (its own included) and
+//               every CTA's (m, l) by asynchronous distributed-shared-memory
+//               stores counted on its mbarrier, then combines them and
+//               writes its slice in bf16.
 // Modes: select only (writes sel / sel_count), attend only (reads them) and
 // full (A-E in one launch, the selection never leaves the chip).  Centroid
 // format (INT4 / BF16) and score aggregation (sum / group max) are template

@@ -101,15 +101,30 @@ def test_traffic_reported_only_for_its_source(monkeypatch, tmp_path):
     assert bench.recorded_traffic() is None
 
 
-def test_kernel_source_hash_follows_the_sources(monkeypatch, tmp_path):
+def test_kernel_source_hash_follows_the_code_not_the_comments(monkeypatch, tmp_path):
     a, b = tmp_path / "a.cu", tmp_path / "b.cuh"
-    a.write_text("kernel A")
-    b.write_text("header")
+    a.write_text('int f(int x) {  // doubles x\n  return 2 * x;\n}\nconst char* s = "a // b";\n')
+    b.write_text("/* header */\n#define N 4\n")
     monkeypatch.setattr(bench, "KERNEL_SOURCES", [str(a), str(b)])
     h0 = bench.kernel_source_hash()
     assert len(h0) == 16
-    a.write_text("kernel A ")                # one byte more: another hash
-    assert bench.kernel_source_hash() != h0
+    # comments, blank lines and indentation: the same code, the same hash
+    a.write_text('// f doubles its argument\n\nint f(int x) {\n    return 2 * x;   /* twice */\n}\n'
+                 'const char* s = "a // b";\n')
+    b.write_text("/* another\n   header */\n#define N 4\n")
+    assert bench.kernel_source_hash() == h0
+    # a token, a string literal's contents or a directive's line: another hash
+    for src_a, src_b in [('int f(int x) { return 3 * x; }\nconst char* s = "a // b";\n', "#define N 4\n"),
+                         ('int f(int x) { return 2 * x; }\nconst char* s = "a // c";\n', "#define N 4\n"),
+                         ('int f(int x) { return 2 * x; }\nconst char* s = "a // b";\n', "#define N 4 int\n")]:
+        a.write_text(src_a)
+        b.write_text(src_b)
+        assert bench.kernel_source_hash() != h0
+
+
+def test_code_text_strips_comments_only():
+    src = 'a = 1; // c1\nb = "/* not a comment */"; /* c2 */ c = \'/\';\n\n  d\t=  2;\n'
+    assert bench.code_text(src) == 'a = 1;\nb = "/* not a comment */"; c = \'/\';\nd = 2;'
 
 
 def test_hbm_peak_measured_else_fallback(monkeypatch, tmp_path):
