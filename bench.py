@@ -151,6 +151,31 @@ def clocks_rejected(clocks) -> list:
     return why
 
 
+def timed_with_clocks(timed, make_sampler, dist=None, device=None):
+    """One timed region with its clock record, timed once more when the
+    record disqualifies it on any rank.
+
+    `timed()` returns the region's max-over-ranks milliseconds; every rank
+    takes the same collective steps, since whether to time again is itself
+    a max over ranks.  Returns (ms, clocks); a second measurement's clocks
+    carry the first under "remeasured_after".
+    """
+    sampler = make_sampler()
+    sampler.start()
+    ms = timed()
+    clocks = sampler.stop()
+    why = clocks_rejected(clocks)
+    if reduce_max(1.0 if why else 0.0, dist, device) > 0:
+        first = {"ms": ms, "why": why, "clocks": clocks}
+        sampler = make_sampler()
+        sampler.start()
+        ms = timed()
+        clocks = sampler.stop()
+        if clocks is not None:
+            clocks["remeasured_after"] = first
+    return ms, clocks
+
+
 def hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -777,22 +802,8 @@ def gpu_arm(args):
         return reduce_max(e0.elapsed_time(e1), dist, dev)
 
     with torch.cuda.stream(stream):
-        sampler = ClockSampler(local)
-        sampler.start()
-        ms = timed(g, args.steps, args.warmup)
-        clocks = sampler.stop()
-        # a region whose clocks disqualify it on any rank is timed once more
-        # on every rank (the decision is itself a max over ranks)
-        why = clocks_rejected(clocks)
-        if reduce_max(1.0 if why else 0.0, dist, dev) > 0:
-            first = {"ms_per_step": ms / args.steps, "why": why,
-                     "clocks": clocks}
-            sampler = ClockSampler(local)
-            sampler.start()
-            ms = timed(g, args.steps, args.warmup)
-            clocks = sampler.stop()
-            if clocks is not None:
-                clocks["remeasured_after"] = first
+        ms, clocks = timed_with_clocks(lambda: timed(g, args.steps, args.warmup),
+                                       lambda: ClockSampler(local), dist, dev)
         ms_plain = timed(g_plain, args.steps, args.warmup)
     for x in layers:
         x.check()
