@@ -172,7 +172,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tensor tile load (no multicast) into this CTA's shared memory.
+// 2-D tensor tile load into this CTA's own shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x,
                                             int y, uint32_t bar) {
     asm volatile(

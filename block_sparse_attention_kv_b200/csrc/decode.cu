@@ -29,7 +29,7 @@
 //   D  attend:  the selected blocks expand to bs/16 pages each; CTA r takes a
 //               contiguous 1/C share of those pages.  Each warp owns every
 //               8th page: it loads the (page, head) K and V slices with 2-D
-//               tensor copies (128-byte swizzle, no multicast) on its own
+//               tensor copies (128-byte swizzle, each CTA's own) on its own
 //               mbarrier into one of its one or two page buffers (two in the
 //               one-CTA-per-SM instance), then computes S^T = Q K^T and O += P V on mma.sync
 //               bf16 tiles with the GQA group as the 16-row M dimension and an
